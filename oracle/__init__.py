@@ -1,0 +1,119 @@
+"""CPU oracle for batched speculative-sampling verification (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or calls it, and this package imports
+nothing from the product.
+
+``verify`` wraps ``sv_oracle.c`` (plain C, double precision); see that file for
+what is computed and which page passage each step follows.  ``build()``
+compiles it with gcc into ``oracle/libsvoracle.so``.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sv_oracle.c")
+_LIB = os.path.join(_HERE, "libsvoracle.so")
+
+ST_TOKEN, ST_ROW, ST_TEMP, ST_RESID0 = 1, 2, 4, 8
+NEAR_ACCEPT, NEAR_CDF = 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (gcc -O2, OpenMP, strict IEEE: no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def load_library(path: str):
+    """Load an oracle shared library built from ``sv_oracle.c`` (or a test variant of it)."""
+    lib = ctypes.CDLL(path)
+    p = ctypes.c_void_p
+    lib.sv_oracle_verify.argtypes = [p, p, ctypes.c_int, p, p, p, p, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int, p, p, p, p, p, p, p,
+                                     ctypes.c_int]
+    lib.sv_oracle_verify.restype = ctypes.c_int
+    lib.sv_oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = load_library(_LIB)
+    return _lib
+
+
+@dataclasses.dataclass
+class OracleResult:
+    out_tokens: np.ndarray   # [B, gamma+1] int32, -1 past the extra token
+    n_accepted: np.ndarray   # [B] int32
+    log_norm: np.ndarray     # [B, 2*gamma+1] float64 (target rows, then draft rows)
+    row_status: np.ndarray   # [B] int32 bitmask
+    near_tie: np.ndarray     # [B] int32 bitmask (1 accept test, 2 inverse CDF)
+    accept_gap: np.ndarray   # [B] float64: min |log u_j - delta_j| over tested j
+    cdf_gap: np.ndarray      # [B] float64: distance of u*S to the chosen bin's edges, / S
+
+
+def max_threads() -> int:
+    return int(_load().sv_oracle_max_threads())
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def verify(target: np.ndarray, draft: np.ndarray, draft_tokens: np.ndarray,
+           temperature: np.ndarray, u_accept: np.ndarray, u_resample: np.ndarray,
+           *, bf16: bool | None = None, n_threads: int = 0, lib=None) -> OracleResult:
+    """Run the oracle.  Logits are float32 arrays, or uint16 bf16 bit patterns."""
+    lib = _load() if lib is None else lib
+    target = np.ascontiguousarray(target)
+    draft = np.ascontiguousarray(draft)
+    if bf16 is None:
+        bf16 = target.dtype == np.uint16
+    want = np.uint16 if bf16 else np.float32
+    if target.dtype != want or draft.dtype != want:
+        raise TypeError("target/draft must both be float32 or both uint16 (bf16 bits)")
+    B, g1, V = target.shape
+    gamma = g1 - 1
+    if draft.shape != (B, gamma, V):
+        raise ValueError("draft shape must be [B, gamma, V]")
+    toks = np.ascontiguousarray(draft_tokens, dtype=np.int32).reshape(B, gamma)
+    T = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    ua = np.ascontiguousarray(u_accept, dtype=np.float32).reshape(B, gamma)
+    ur = np.ascontiguousarray(u_resample, dtype=np.float32).reshape(B)
+    out_t = np.empty((B, gamma + 1), dtype=np.int32)
+    out_n = np.empty((B,), dtype=np.int32)
+    ln = np.empty((B, 2 * gamma + 1), dtype=np.float64)
+    st = np.empty((B,), dtype=np.int32)
+    nr = np.empty((B,), dtype=np.int32)
+    ag = np.empty((B,), dtype=np.float64)
+    cg = np.empty((B,), dtype=np.float64)
+    rc = lib.sv_oracle_verify(_ptr(target), _ptr(draft), int(bool(bf16)), _ptr(toks), _ptr(T),
+                              _ptr(ua), _ptr(ur), B, gamma, V, _ptr(out_t), _ptr(out_n),
+                              _ptr(ln), _ptr(st), _ptr(nr), _ptr(ag), _ptr(cg), int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"sv_oracle_verify failed ({rc})")
+    return OracleResult(out_t, out_n, ln, st, nr, ag, cg)
+
+
+def verify_workload(w, n_threads: int = 0) -> OracleResult:
+    """Run the oracle on a ``Workload`` from the seeded generators."""
+    return verify(w.target, w.draft, w.draft_tokens, w.temperature, w.u_accept, w.u_resample,
+                  bf16=(w.dtype == "bf16"), n_threads=n_threads)

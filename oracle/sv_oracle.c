@@ -1,0 +1,282 @@
+/*
+ * sv_oracle.c -- plain, slow, double-precision CPU oracle for batched
+ * speculative-sampling verification.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg use this file.  It shares no code, header or constant with
+ * the CUDA library; the product path never calls it.
+ *
+ * What it computes, per sequence b (sources named in brackets):
+ *
+ *  1. Temperature before log-softmax, in log space [FlashSpec, Metodologia 1,
+ *     "Estabilidade Numerica"; Significancia, engineering lessons]:
+ *        lse(row) = M/T + log sum_v exp((l_v - M)/T),  M = max_v l_v
+ *     for every target row j in [0, gamma] and draft row j in [0, gamma).
+ *  2. The per-candidate test on two log-probability scalars [FlashSpec,
+ *     Metodologia 1, "Mecanismo"]:
+ *        log p_j(x_j) = lt[j][x_j]/T - lse_t[j],  log q_j(x_j) = ld[j][x_j]/T - lse_d[j]
+ *        accept j  iff  log u_j < log p_j(x_j) - log q_j(x_j)
+ *     The accepted prefix ends at the first rejection n; the rest is dropped
+ *     [Speculative Speculative Decoding, "O Essencial", step 3].
+ *  3. The verification outcome is (number accepted, one more token)
+ *     [Speculative Speculative Decoding, Metodologia 2, "Conceito Central" 1].
+ *     After a rejection at n the extra token comes from the residual
+ *     distribution norm(max(0, p_n - q_n)) [same page, Desafios 2, "Amostragem
+ *     Saguaro"]; when all gamma drafts are accepted it is the bonus token drawn
+ *     from the target's (gamma+1)-th distribution p_gamma.
+ *     Inverse CDF: the token is the smallest k with C_k > u * S, where C_k is the
+ *     running sum of the weights and S their total; if rounding leaves no such k,
+ *     the last k with a positive weight.  If the residual is all zero, the draw
+ *     falls back to p_n (row-status bit 8).
+ *  4. T == 0 is greedy verification: accept j iff x_j is the first argmax of
+ *     target row j; the extra token is the first argmax of target row n.  The
+ *     draft logits and the uniforms are not used.
+ *
+ * The pages print neither min(1, p/q), the residual nor the bonus rule; the
+ * formulas above are the standard speculative-sampling rule whose output
+ * distribution equals the target's, which is the property the pages require
+ * [FlashSpec, Metodologia 2, "Garantia Teorica"; Significancia, Teorema 1].
+ *
+ * Contract details that the pages leave open (library readings):
+ *   - valid temperature: T == 0, or T finite and >= 1e-6; otherwise status 4;
+ *   - status 1: some draft token outside [0, V);
+ *   - status 2: a row that is read holds NaN or +inf, or is all -inf
+ *     (T > 0: all 2*gamma+1 rows; T == 0: the gamma+1 target rows);
+ *   - with status 1, 2 or 4 the sequence emits n = 0 and all tokens -1;
+ *   - tokens past the extra one are -1;
+ *   - log_norm is NaN for greedy sequences, invalid T and bad rows.
+ *
+ * Near-tie report (for comparing an implementation that rounds differently):
+ *   bit 1: |log u_j - delta_j| < 1e-6 at some tested position j;
+ *   bit 2: at the chosen token k, min(|C_{k-1} - uS|, |C_k - uS|) / S < 1e-6.
+ *
+ * Inputs: logits are float32, or bf16 given as uint16 bit patterns; every
+ * value is widened exactly to double before any arithmetic.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_T_MIN 1e-6
+#define ORACLE_NEAR 1e-6
+
+enum { ST_TOKEN = 1, ST_ROW = 2, ST_TEMP = 4, ST_RESID0 = 8 };
+enum { NEAR_ACCEPT = 1, NEAR_CDF = 2 };
+
+static double widen(const void* base, int is_bf16, size_t i)
+{
+    if (!is_bf16) return (double)((const float*)base)[i];
+    uint32_t bits = (uint32_t)((const uint16_t*)base)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* One row's log-normaliser of l/T.  Returns 0 if the row is bad. */
+static int row_lse(const void* base, int is_bf16, size_t off, int V, double T, double* lse)
+{
+    double M = -INFINITY;
+    for (int v = 0; v < V; ++v) {
+        double l = widen(base, is_bf16, off + (size_t)v);
+        if (isnan(l)) return 0;
+        if (l > M) M = l;
+    }
+    if (isinf(M)) return 0; /* +inf present, or every entry -inf */
+    double s = 0.0;
+    for (int v = 0; v < V; ++v) s += exp((widen(base, is_bf16, off + (size_t)v) - M) / T);
+    *lse = M / T + log(s);
+    return 1;
+}
+
+/* First index of the largest value.  Returns -1 if the row is bad. */
+static int row_argmax(const void* base, int is_bf16, size_t off, int V)
+{
+    double best = -INFINITY;
+    int arg = -1;
+    for (int v = 0; v < V; ++v) {
+        double l = widen(base, is_bf16, off + (size_t)v);
+        if (isnan(l)) return -1;
+        if (l > best) { best = l; arg = v; }
+    }
+    if (arg < 0 || isinf(best)) return -1;
+    return arg;
+}
+
+/* Smallest k with running sum C_k > u*S; if none, the last k with w_k > 0. */
+static int inverse_cdf(const double* w, int V, double u, int* near, double* gap)
+{
+    double S = 0.0;
+    for (int v = 0; v < V; ++v) S += w[v];
+    double target = u * S;
+    double C = 0.0, prev = 0.0;
+    int k = -1;
+    for (int v = 0; v < V; ++v) {
+        prev = C;
+        C += w[v];
+        if (C > target) { k = v; break; }
+    }
+    if (k < 0) {
+        for (int v = V - 1; v >= 0; --v)
+            if (w[v] > 0.0) { k = v; break; }
+        *near |= NEAR_CDF;
+        *gap = 0.0;
+        return k;
+    }
+    *gap = fmin(fabs(prev - target), fabs(C - target)) / S;
+    if (*gap < ORACLE_NEAR) *near |= NEAR_CDF;
+    return k;
+}
+
+static void verify_one(const void* tgt, const void* dft, int is_bf16, const int32_t* tok,
+                       double T, const float* u_acc, double u_res, int gamma, int V, size_t b,
+                       int32_t* out_tok, int32_t* out_n, double* lnorm, int32_t* status,
+                       int32_t* near, double* agap, double* cgap, double* wbuf)
+{
+    const int R = 2 * gamma + 1;
+    int st = 0, nr = 0;
+    *agap = INFINITY;
+    *cgap = INFINITY;
+    for (int j = 0; j <= gamma; ++j) out_tok[j] = -1;
+    for (int r = 0; r < R; ++r) lnorm[r] = NAN;
+    *out_n = 0;
+
+    if (!(T == 0.0 || (isfinite(T) && T >= ORACLE_T_MIN))) {
+        *status = ST_TEMP;
+        *near = 0;
+        return;
+    }
+    for (int j = 0; j < gamma; ++j)
+        if (tok[j] < 0 || tok[j] >= V) st |= ST_TOKEN;
+
+    const size_t trow0 = b * (size_t)(gamma + 1) * (size_t)V;
+    const size_t drow0 = b * (size_t)gamma * (size_t)V;
+
+    if (T == 0.0) {
+        int arg[64];
+        for (int j = 0; j <= gamma; ++j) {
+            arg[j] = row_argmax(tgt, is_bf16, trow0 + (size_t)j * V, V);
+            if (arg[j] < 0) st |= ST_ROW;
+        }
+        if (st) { *status = st; *near = 0; return; }
+        int n = gamma;
+        for (int j = 0; j < gamma; ++j)
+            if (tok[j] != arg[j]) { n = j; break; }
+        for (int j = 0; j < n; ++j) out_tok[j] = tok[j];
+        out_tok[n] = arg[n];
+        *out_n = n;
+        *status = 0;
+        *near = 0;
+        return;
+    }
+
+    double lse_t[33], lse_d[32];
+    for (int j = 0; j <= gamma; ++j) {
+        if (row_lse(tgt, is_bf16, trow0 + (size_t)j * V, V, T, &lse_t[j])) lnorm[j] = lse_t[j];
+        else st |= ST_ROW;
+    }
+    for (int j = 0; j < gamma; ++j) {
+        if (row_lse(dft, is_bf16, drow0 + (size_t)j * V, V, T, &lse_d[j])) lnorm[gamma + 1 + j] = lse_d[j];
+        else st |= ST_ROW;
+    }
+    if (st) { /* good rows keep their log_norm; the sequence emits nothing */
+        *status = st;
+        *near = 0;
+        return;
+    }
+
+    /* accept scan in log space */
+    int n = gamma;
+    for (int j = 0; j < gamma; ++j) {
+        double lp = widen(tgt, is_bf16, trow0 + (size_t)j * V + (size_t)tok[j]) / T - lse_t[j];
+        double lq = widen(dft, is_bf16, drow0 + (size_t)j * V + (size_t)tok[j]) / T - lse_d[j];
+        double delta = lp - lq;
+        double lu = log((double)u_acc[j]);
+        if (fabs(lu - delta) < *agap) *agap = fabs(lu - delta);
+        if (fabs(lu - delta) < ORACLE_NEAR) nr |= NEAR_ACCEPT;
+        if (!(lu < delta)) { n = j; break; }
+    }
+
+    int k;
+    if (n < gamma) {
+        double S = 0.0;
+        for (int v = 0; v < V; ++v) {
+            double p = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);
+            double q = exp(widen(dft, is_bf16, drow0 + (size_t)n * V + v) / T - lse_d[n]);
+            wbuf[v] = fmax(0.0, p - q);
+            S += wbuf[v];
+        }
+        if (!(S > 0.0)) {
+            st |= ST_RESID0;
+            for (int v = 0; v < V; ++v)
+                wbuf[v] = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);
+        }
+        k = inverse_cdf(wbuf, V, u_res, &nr, cgap);
+    } else {
+        for (int v = 0; v < V; ++v)
+            wbuf[v] = exp(widen(tgt, is_bf16, trow0 + (size_t)gamma * V + v) / T - lse_t[gamma]);
+        k = inverse_cdf(wbuf, V, u_res, &nr, cgap);
+    }
+    for (int j = 0; j < n; ++j) out_tok[j] = tok[j];
+    out_tok[n] = k;
+    *out_n = n;
+    *status = st;
+    *near = nr;
+}
+
+/*
+ * target: [B][gamma+1][V], draft: [B][gamma][V]; is_bf16 selects uint16 bf16 bits.
+ * Outputs: out_tokens [B][gamma+1], out_n [B], log_norm [B][2*gamma+1],
+ * row_status [B], near_tie [B], accept_gap [B] (smallest |log u_j - delta_j| over
+ * the tested positions), cdf_gap [B] (the inverse-CDF gap above; +inf when no draw
+ * was made).  Returns 0, or -1 on a bad shape.
+ */
+int sv_oracle_verify(const void* target, const void* draft, int is_bf16,
+                     const int32_t* draft_tokens, const float* temperature,
+                     const float* u_accept, const float* u_resample,
+                     int B, int gamma, int V,
+                     int32_t* out_tokens, int32_t* out_n, double* log_norm,
+                     int32_t* row_status, int32_t* near_tie, double* accept_gap,
+                     double* cdf_gap, int n_threads)
+{
+    if (B < 0 || gamma < 1 || gamma > 32 || V < 1) return -1;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        double* wbuf = (double*)malloc(sizeof(double) * (size_t)V);
+        if (!wbuf) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b) {
+            if (!wbuf) continue;
+            verify_one(target, draft, is_bf16, draft_tokens + (size_t)b * gamma,
+                       (double)temperature[b], u_accept + (size_t)b * gamma,
+                       (double)u_resample[b], gamma, V, (size_t)b,
+                       out_tokens + (size_t)b * (gamma + 1), out_n + b,
+                       log_norm + (size_t)b * (2 * gamma + 1), row_status + b, near_tie + b,
+                       accept_gap + b, cdf_gap + b, wbuf);
+        }
+        free(wbuf);
+    }
+    return failed ? -2 : 0;
+}
+
+/* Number of threads an OpenMP region would use (for reporting). */
+int sv_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

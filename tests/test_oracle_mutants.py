@@ -1,0 +1,75 @@
+"""Each planted mistake in a copy of the oracle must fail at least one pin.
+
+The copies are made by text substitution of ``oracle/sv_oracle.c`` into a
+temporary directory and compiled there; the real oracle is never modified.
+This shows the pins are sharp enough to catch a dropped term, a wrong sign, a
+wrong index or a transposed step anywhere on the path."""
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "sv_oracle.c")
+
+MUTANTS = {
+    "temperature_after_log_softmax": (
+        "s += exp((widen(base, is_bf16, off + (size_t)v) - M) / T);\n    *lse = M / T + log(s);",
+        "s += exp(widen(base, is_bf16, off + (size_t)v) - M);\n    *lse = (M + log(s)) / T;"),
+    "residual_sign_flipped": ("wbuf[v] = fmax(0.0, p - q);", "wbuf[v] = fmax(0.0, q - p);"),
+    "residual_not_clamped": ("wbuf[v] = fmax(0.0, p - q);", "wbuf[v] = p - q;"),
+    "linear_uniform_in_log_test": ("double lu = log((double)u_acc[j]);", "double lu = (double)u_acc[j];"),
+    "gather_without_temperature": ("/ T - lse_t[j];", "- lse_t[j];"),
+    "residual_from_next_position": (
+        "double p = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);",
+        "double p = exp(widen(tgt, is_bf16, trow0 + (size_t)(n + 1) * V + v) / T - lse_t[n + 1]);"),
+    "bonus_from_wrong_row": (
+        "trow0 + (size_t)gamma * V + v) / T - lse_t[gamma]);",
+        "trow0 + (size_t)(gamma - 1) * V + v) / T - lse_t[gamma - 1]);"),
+    "greedy_last_argmax": ("if (l > best) { best = l; arg = v; }", "if (l >= best) { best = l; arg = v; }"),
+    "scan_past_first_rejection": ("if (!(lu < delta)) { n = j; break; }", "if (!(lu < delta)) { n = j; }"),
+    "cdf_not_scaled_by_total": ("double target = u * S;", "double target = u;"),
+    "draft_normaliser_for_target": (
+        "double lp = widen(tgt, is_bf16, trow0 + (size_t)j * V + (size_t)tok[j]) / T - lse_t[j];",
+        "double lp = widen(tgt, is_bf16, trow0 + (size_t)j * V + (size_t)tok[j]) / T - lse_d[j];"),
+}
+
+
+def _build_mutant(name, tmpdir):
+    src = open(SRC).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    path = os.path.join(tmpdir, f"{name}.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    so = os.path.join(tmpdir, f"lib_{name}.so")
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", so, path, "-lm"])
+    return oracle.load_library(so)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    with tempfile.TemporaryDirectory() as d:
+        lib = _build_mutant(name, d)
+
+        def verify(*a, **k):
+            return oracle.verify(*a, lib=lib, **k)
+
+        caught = []
+        for check in P.ALL_ORACLE_CHECKS:
+            try:
+                with np.errstate(all="ignore"):
+                    check(verify)
+            except Exception as e:  # noqa: BLE001 - any failure counts as caught
+                caught.append((check.__name__, type(e).__name__))
+                break
+        if not caught:
+            try:
+                P.check_bonus_distribution(verify, min_samples=3000)
+            except Exception as e:  # noqa: BLE001
+                caught.append(("check_bonus_distribution", type(e).__name__))
+        assert caught, f"planted mistake {name} passed every pin"
