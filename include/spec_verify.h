@@ -1,0 +1,140 @@
+/*
+ * spec_verify.h -- C ABI of the B200 batched speculative-sampling verifier.
+ *
+ * One call verifies B independent sequences, each carrying gamma draft tokens,
+ * entirely on the GPU with no host synchronisation.  The on-device accept /
+ * reject decision replaces a per-step device-to-host copy whose cost grows with
+ * the vocabulary size [FlashSpec (gist.science rs-10162738), "Declaracao do
+ * Problema" 1 and Metodologia 1, "Kernel de Verificacao no Dispositivo"].
+ *
+ * For every sequence b with temperature T = temperature[b] > 0:
+ *   1. Both models' logits are scaled by 1/T before the log-softmax, and every
+ *      row is normalised in log space over the whole vocabulary V in one
+ *      streaming pass [FlashSpec, Metodologia 1, "Estabilidade Numerica";
+ *      "Significancia", engineering lessons]:
+ *          lse(row) = log sum_v exp(l_v / T)
+ *   2. For each draft position j the kernel reads two log-probability scalars,
+ *          log p_j(x_j) = lt[b][j][x_j]/T - lse_t[j],
+ *          log q_j(x_j) = ld[b][j][x_j]/T - lse_d[j]
+ *      [FlashSpec, Metodologia 1, "Mecanismo"], and accepts x_j iff
+ *          log u_accept[b][j] < log p_j(x_j) - log q_j(x_j).
+ *      The accepted prefix ends at the first rejection n (n = gamma if none)
+ *      and the rest of the draft is dropped [Speculative Speculative Decoding
+ *      (gist.science 2603.03251), "O Essencial", step 3].
+ *   3. The outcome is n plus one more token [Speculative Speculative Decoding,
+ *      Metodologia 2, "Conceito Central" 1]: after a rejection it is drawn from
+ *      the residual distribution norm(max(0, p_n - q_n)) [same page, Desafios 2,
+ *      "Amostragem Saguaro"]; after gamma acceptances it is the bonus token,
+ *      drawn from the target's (gamma+1)-th distribution p_gamma.  The draw is
+ *      an inverse CDF with u = u_resample[b]: the smallest token k whose running
+ *      weight sum C_k exceeds u * (sum of all weights).
+ * With T == 0 the step is greedy: x_j is accepted iff it is the first argmax of
+ * target row j, and the extra token is the first argmax of target row n.  The
+ * draft logits and the uniforms of such a sequence are not read.
+ *
+ * The uniforms are inputs, so a call is a deterministic function of its
+ * arguments and can be reproduced bit for bit.
+ *
+ * Numerics: the normaliser sums are accumulated in fp32 from exact bf16/fp32
+ * inputs and finished in fp64; the accept test runs in fp64.  Compared with an
+ * exact evaluation, a decision can differ only when |log u - (log p - log q)|
+ * or the inverse-CDF gap to u is below ~1e-6.
+ */
+#ifndef SPEC_VERIFY_H_
+#define SPEC_VERIFY_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so C callers need no CUDA header. */
+struct CUstream_st;
+
+typedef enum {
+    SV_OK = 0,
+    SV_ERR_INVALID_ARG = 1,        /* bad size, null required pointer, bad enum */
+    SV_ERR_UNSUPPORTED_DTYPE = 2,  /* dt is not SV_DTYPE_F32 / SV_DTYPE_BF16 */
+    SV_ERR_MISALIGNED = 3,         /* logits not 16-byte aligned, or a pointer not
+                                      aligned to its element / workspace to 256 bytes */
+    SV_ERR_WORKSPACE_TOO_SMALL = 4,/* workspace_bytes < spec_verify_workspace_size() */
+    SV_ERR_CUDA = 5                /* a CUDA launch or runtime call failed */
+} sv_status;
+
+typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
+
+/* Limits checked on the host before anything is launched. */
+#define SV_MAX_GAMMA 32
+#define SV_MAX_V (1 << 30)
+/* Smallest positive temperature; 0 < T < SV_TEMPERATURE_MIN counts as invalid. */
+#define SV_TEMPERATURE_MIN 1e-6f
+
+/* Per-sequence status bits written to out_row_status (data-dependent errors
+ * never trap; they are reported here).  With bit 1, 2 or 4 the sequence emits
+ * n_accepted = 0 and out_tokens all -1. */
+#define SV_ROW_BAD_TOKEN 1        /* some draft token outside [0, V) */
+#define SV_ROW_BAD_LOGITS 2       /* a row that is read holds NaN or +inf, or is all -inf */
+#define SV_ROW_BAD_TEMPERATURE 4  /* T < 0, NaN, +inf, or 0 < T < SV_TEMPERATURE_MIN */
+#define SV_ROW_RESIDUAL_ZERO 8    /* residual mass was 0; the token was drawn from p_n */
+
+/*
+ * Bytes of device workspace spec_verify() needs for this shape (0 on a bad
+ * shape).  The workspace is caller-owned device memory, 256-byte aligned.
+ *
+ * Its first 8*B bytes are completion counters that must be zero when a call
+ * starts.  Zero the whole workspace once after allocating it (for example with
+ * spec_verify_workspace_init); every call that runs to completion leaves the
+ * counters at zero again, so one workspace serves any number of calls with the
+ * same (B, gamma, V, dt).  Zero it again before reusing it for another shape.
+ * Calls that share a workspace must be ordered (same stream, or events).
+ */
+size_t spec_verify_workspace_size(int B, int gamma, int V, sv_dtype dt);
+
+/* cudaMemsetAsync(workspace, 0, workspace_bytes, stream). */
+sv_status spec_verify_workspace_init(void* workspace, size_t workspace_bytes,
+                                     struct CUstream_st* stream);
+
+/*
+ * Verify B sequences.  All pointers are caller-owned DEVICE memory on the
+ * current device; the library allocates nothing, keeps no state between calls
+ * and does not synchronise with the host.  Work is enqueued on `stream` and the
+ * call returns right after the enqueue; results are visible to later work on
+ * that stream.
+ *
+ *   target_logits   [B][gamma+1][V] of dt, contiguous, 16-byte aligned
+ *   draft_logits    [B][gamma][V]   of dt, contiguous, 16-byte aligned
+ *   draft_tokens    [B][gamma] int32
+ *   temperature     [B] float; 0 = greedy
+ *   u_accept        [B][gamma] float, expected in (0, 1)
+ *   u_resample      [B] float, expected in (0, 1)
+ *   out_tokens      [B][gamma+1] int32: the n accepted drafts, the extra token,
+ *                   then -1
+ *   out_n_accepted  [B] int32 in [0, gamma]
+ *   workspace       see spec_verify_workspace_size()
+ *   out_log_norm    optional [B][2*gamma+1] double: lse of the target rows, then
+ *                   the draft rows; NaN for greedy or invalid sequences and bad rows
+ *   out_row_status  optional [B] int32 bitmask of SV_ROW_* (0 = ok)
+ *
+ * Returns SV_OK after a successful enqueue.  Host-checkable errors return before
+ * anything is launched and leave every output untouched.  SV_ERR_CUDA reports a
+ * failed launch; outputs are then undefined.
+ */
+sv_status spec_verify(const void* target_logits, const void* draft_logits, sv_dtype dt,
+                      const int32_t* draft_tokens, const float* temperature,
+                      const float* u_accept, const float* u_resample,
+                      int32_t* out_tokens, int32_t* out_n_accepted,
+                      int B, int gamma, int V,
+                      void* workspace, size_t workspace_bytes,
+                      double* out_log_norm, int32_t* out_row_status,
+                      struct CUstream_st* stream);
+
+/* Static description of a status code; never NULL. */
+const char* spec_verify_status_string(sv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEC_VERIFY_H_ */

@@ -1,0 +1,170 @@
+"""Thin ctypes binding over the C ABI in ``include/spec_verify.h``.
+
+Argument marshalling only: every step of verification runs in the CUDA
+kernels of ``lib/libspecverify.so``.  Torch supplies device memory and the
+current stream.  There is no fallback: if the library is missing or the
+tensors are not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libspecverify.so")
+
+SV_OK = 0
+SV_DTYPE_F32, SV_DTYPE_BF16 = 0, 1
+ROW_BAD_TOKEN, ROW_BAD_LOGITS, ROW_BAD_TEMPERATURE, ROW_RESIDUAL_ZERO = 1, 2, 4, 8
+EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_init",
+            "spec_verify_status_string")
+
+_lib = None
+
+
+class SpecVerifyError(ValueError):
+    """A non-OK status returned by the C ABI."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(f"spec_verify status {status}: {message}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the C-ABI library and declare its signatures (raises if it is missing)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} (run __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.spec_verify_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.spec_verify_workspace_size.restype = sz
+    lib.spec_verify_workspace_init.argtypes = [vp, sz, vp]
+    lib.spec_verify_workspace_init.restype = i32
+    lib.spec_verify.argtypes = [vp, vp, i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, vp, vp, vp]
+    lib.spec_verify.restype = i32
+    lib.spec_verify_status_string.argtypes = [i32]
+    lib.spec_verify_status_string.restype = ctypes.c_char_p
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().spec_verify_status_string(int(status)).decode()
+
+
+def _dt_code(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return SV_DTYPE_F32
+    if dtype == torch.bfloat16:
+        return SV_DTYPE_BF16
+    raise TypeError(f"logits dtype must be float32 or bfloat16, got {dtype}")
+
+
+def workspace_size(B: int, gamma: int, V: int, dtype: torch.dtype) -> int:
+    return int(load_library().spec_verify_workspace_size(B, gamma, V, _dt_code(dtype)))
+
+
+_ws_cache: Dict[Tuple, torch.Tensor] = {}
+
+
+def workspace_for(B: int, gamma: int, V: int, dtype: torch.dtype, device) -> torch.Tensor:
+    """A zero-initialised workspace cached per (device, shape).  Calls that share it
+    must be ordered on one stream; pass ``workspace=`` to run shapes concurrently."""
+    device = torch.device(device)
+    key = (device.index, B, gamma, V, dtype)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(max(1, workspace_size(B, gamma, V, dtype)), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _check(t: torch.Tensor, name: str, dtype, shape, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Tensor,
+           temperature: torch.Tensor, u_accept: torch.Tensor, u_resample: torch.Tensor, *,
+           return_log_norm: bool = False, return_row_status: bool = False,
+           out_tokens: torch.Tensor | None = None, out_n_accepted: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """Verify B sequences on the GPU (see include/spec_verify.h for the rule).
+
+    target [B, gamma+1, V] and draft [B, gamma, V] (float32 or bfloat16),
+    draft_tokens [B, gamma] int32, temperature [B] float32 (0 = greedy),
+    u_accept [B, gamma] and u_resample [B] float32 in (0, 1), all on one CUDA device.
+    Returns (out_tokens [B, gamma+1] int32, n_accepted [B] int32) plus, if asked,
+    log_norm [B, 2*gamma+1] float64 and row_status [B] int32.  Runs asynchronously on
+    the current stream (or ``stream``); raises SpecVerifyError on a non-OK status."""
+    lib = load_library()
+    if not isinstance(target, torch.Tensor) or target.device.type != "cuda":
+        raise ValueError("target must be a CUDA tensor")
+    device = target.device
+    if target.dim() != 3:
+        raise ValueError("target must be [B, gamma+1, V]")
+    B, g1, V = target.shape
+    gamma = g1 - 1
+    dt = _dt_code(target.dtype)
+    _check(target, "target", None, (B, gamma + 1, V), device)
+    _check(draft, "draft", target.dtype, (B, gamma, V), device)
+    _check(draft_tokens, "draft_tokens", torch.int32, (B, gamma), device)
+    _check(temperature, "temperature", torch.float32, (B,), device)
+    _check(u_accept, "u_accept", torch.float32, (B, gamma), device)
+    _check(u_resample, "u_resample", torch.float32, (B,), device)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, gamma + 1), dtype=torch.int32, device=device)
+    if out_n_accepted is None:
+        out_n_accepted = torch.empty((B,), dtype=torch.int32, device=device)
+    _check(out_tokens, "out_tokens", torch.int32, (B, gamma + 1), device)
+    _check(out_n_accepted, "out_n_accepted", torch.int32, (B,), device)
+    log_norm = torch.empty((B, 2 * gamma + 1), dtype=torch.float64, device=device) if return_log_norm else None
+    row_status = torch.empty((B,), dtype=torch.int32, device=device) if return_row_status else None
+    if workspace is None:
+        workspace = workspace_for(B, gamma, V, target.dtype, device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        st = lib.spec_verify(target.data_ptr(), draft.data_ptr(), dt, draft_tokens.data_ptr(),
+                             temperature.data_ptr(), u_accept.data_ptr(), u_resample.data_ptr(),
+                             out_tokens.data_ptr(), out_n_accepted.data_ptr(), B, gamma, V,
+                             workspace.data_ptr(), workspace.numel(),
+                             log_norm.data_ptr() if log_norm is not None else None,
+                             row_status.data_ptr() if row_status is not None else None,
+                             s.cuda_stream)
+    if st != SV_OK:
+        raise SpecVerifyError(st, status_string(st))
+    out = [out_tokens, out_n_accepted]
+    if return_log_norm:
+        out.append(log_norm)
+    if return_row_status:
+        out.append(row_status)
+    return tuple(out)
+
+
+def to_device(w, device="cuda"):
+    """Copy a ``workloads.Workload`` (numpy) to torch tensors on ``device``."""
+    def logits(a):
+        t = torch.from_numpy(a)
+        if w.dtype == "bf16":
+            t = t.view(torch.bfloat16)
+        return t.to(device)
+    return dict(target=logits(w.target), draft=logits(w.draft),
+                draft_tokens=torch.from_numpy(w.draft_tokens).to(device),
+                temperature=torch.from_numpy(w.temperature).to(device),
+                u_accept=torch.from_numpy(w.u_accept).to(device),
+                u_resample=torch.from_numpy(w.u_resample).to(device))

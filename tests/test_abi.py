@@ -1,0 +1,78 @@
+"""The C-ABI library loads and exports every function that include/*.h declares
+(no GPU needed: nothing is called that touches the device)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from speculative_decoding_verification_84_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*?[\s\*]+([a-z_][a-z0-9_]*)\s*\(",
+                             text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def test_header_declares_expected_api():
+    assert set(binding.EXPORTED) <= _declared_functions()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in sorted(_declared_functions()):
+        assert hasattr(lib, name), f"{name} missing from {build.LIB}"
+        getattr(lib, name)  # resolves via dlsym
+
+
+def test_nm_lists_symbols(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True).stdout
+    for name in _declared_functions():
+        assert re.search(rf"\bT {name}$", out, flags=re.M), name
+
+
+def test_workspace_size_host_only(lib):
+    s = binding.workspace_size(64, 5, 128256, __import__("torch").bfloat16)
+    assert s > 0 and s % 256 == 0
+    assert lib.spec_verify_workspace_size(0, 5, 100, 0) == 0
+    assert lib.spec_verify_workspace_size(4, 0, 100, 0) == 0
+    assert lib.spec_verify_workspace_size(4, 33, 100, 0) == 0
+    assert lib.spec_verify_workspace_size(4, 2, 0, 0) == 0
+    assert lib.spec_verify_workspace_size(4, 2, 100, 7) == 0
+
+
+def test_host_validation_before_launch(lib):
+    """Host-checkable errors return before any CUDA call (safe without a GPU)."""
+    vp = ctypes.c_void_p
+    good = vp(1 << 20)
+    ws_size = lib.spec_verify_workspace_size(2, 2, 64, 0)
+    args = [good, good, 0, good, good, good, good, good, good, 2, 2, 64, good, ws_size, None, None, None]
+    bad_dtype = list(args); bad_dtype[2] = 5
+    assert lib.spec_verify(*bad_dtype) == 2
+    bad_b = list(args); bad_b[9] = 0
+    assert lib.spec_verify(*bad_b) == 1
+    bad_g = list(args); bad_g[10] = 40
+    assert lib.spec_verify(*bad_g) == 1
+    null = list(args); null[0] = None
+    assert lib.spec_verify(*null) == 1
+    mis = list(args); mis[0] = vp((1 << 20) + 8)
+    assert lib.spec_verify(*mis) == 3
+    small = list(args); small[13] = ws_size - 1
+    assert lib.spec_verify(*small) == 4
+    for s in range(6):
+        assert lib.spec_verify_status_string(s)

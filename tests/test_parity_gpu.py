@@ -1,0 +1,146 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Bar: n_accepted / out_tokens bit-exact except sequences within 1e-6 of a
+decision boundary (counted); per-row log-normaliser within 1e-5 relative;
+row status exact.  See parity.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from speculative_decoding_verification_84_b200 import binding, workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _report(name, stats):
+    print(f"[parity] {name}: {stats}")
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c5"])
+def test_config_full(name):
+    """Whole configuration, every sequence compared."""
+    w = W.make_workload(name)
+    g = parity.run_gpu(w)
+    st = parity.compare(g, oracle.verify_workload(w))
+    _report(name, st)
+    parity.assert_parity(st)
+
+
+def test_config_c4_full_size_sampled():
+    """c4 at full size (B=256, gamma=8, V=151936) on the GPU; the oracle checks a
+    sample of sequences from every temperature class (greedy, 0.6, 1.0)."""
+    w = W.make_workload("c4")
+    g = parity.run_gpu(w)
+    idx = list(range(0, 256, 7)) + [253, 254, 255]
+    st = parity.compare(g, oracle.verify_workload(w.subset(idx)), idx=np.array(idx))
+    _report("c4", st)
+    parity.assert_parity(st)
+
+
+RAGGED = [
+    (1, 1, 1, "f32"), (3, 2, 7, "bf16"), (5, 3, 9, "f32"), (2, 7, 1000, "bf16"), (4, 1, 1025, "f32"),
+    (3, 4, 4097, "bf16"), (17, 5, 3001, "bf16"), (2, 32, 333, "f32"), (6, 3, 33333, "bf16"),
+    (1, 4, 32003, "f32"), (9, 2, 8195, "f32"), (40, 2, 257, "bf16"),
+]
+
+
+@pytest.mark.parametrize("B,gamma,V,dt", RAGGED)
+def test_ragged_shapes(B, gamma, V, dt):
+    """Odd vocabulary sizes (misaligned rows, ragged tails), gamma 1..32, mixed T incl. greedy."""
+    T = np.array([0.0, 0.4, 1.0, 1.7, 1e-3][: 5] * ((B + 4) // 5), np.float32)[:B]
+    w = W.make_random(B, gamma, V, dt, seed=1000 + V + 7 * B + gamma, T=T)
+    st = parity.compare(parity.run_gpu(w), oracle.verify_workload(w))
+    _report(f"{B}x{gamma}x{V}-{dt}", st)
+    parity.assert_parity(st)
+
+
+def test_edge_cases():
+    """NaN / +inf / all -inf rows, out-of-range tokens, invalid temperatures, masked vocab."""
+    rng = np.random.default_rng(9)
+    B, gamma, V = 14, 3, 300
+    tgt = (rng.standard_normal((B, gamma + 1, V)) * 2).astype(np.float32)
+    dft = (tgt[:, :gamma] + rng.standard_normal((B, gamma, V))).astype(np.float32)
+    toks = rng.integers(0, V, (B, gamma)).astype(np.int32)
+    T = np.ones(B, np.float32)
+    tgt[0, 1, 17] = np.nan
+    tgt[1, 2, 5] = np.inf
+    dft[2, 0, :] = -np.inf
+    toks[3, 1] = V
+    toks[4, 0] = -5
+    T[5], T[6], T[7], T[8] = -1.0, np.nan, np.inf, 1e-8
+    T[9] = 0.0
+    dft[9, :, :] = np.nan                      # greedy never reads the draft
+    tgt[10, :, ::3] = -np.inf                  # masked vocabulary
+    dft[10, :, 1::3] = -np.inf
+    T[11] = 0.0
+    tgt[11, 0, :] = 1.0                        # all-tie greedy row: index 0 wins
+    toks[11, 0] = 0
+    tgt[12, 0, :] = -np.inf                    # all -inf row
+    w = W.Workload("edges", "f32", tgt, dft, toks, T, W.draw_uniforms(rng, (B, gamma)),
+                   W.draw_uniforms(rng, (B,)))
+    ref = oracle.verify_workload(w)
+    assert ref.row_status[:9].tolist() == [2, 2, 2, 1, 1, 4, 4, 4, 4]
+    st = parity.compare(parity.run_gpu(w), ref)
+    _report("edges", st)
+    parity.assert_parity(st)
+
+
+def test_golden_worked_example_gpu():
+    import golden_cases
+    fx, a = golden_cases.worked_example_v4()
+    d = {k: torch.from_numpy(v).cuda() for k, v in a.items()}
+    toks, n = binding.verify(**d)
+    for i, c in enumerate(fx["cases"]):
+        assert int(n[i]) == c["expect_n"], c["derivation"]
+        assert toks[i].tolist() == c["expect_tokens"], c["derivation"]
+
+
+def test_deterministic_and_workspace_reuse():
+    """Same inputs -> identical outputs over repeated calls on one workspace (the
+    completion counters reset themselves)."""
+    w = W.make_workload("c2")
+    d = binding.to_device(w)
+    first = [t.clone() for t in binding.verify(**d, return_log_norm=True)]
+    for _ in range(5):
+        again = binding.verify(**d, return_log_norm=True)
+        for x, y in zip(first, again):
+            assert torch.equal(x, y)
+
+
+def test_host_errors_leave_outputs_untouched():
+    w = W.make_random(2, 2, 64, "f32", seed=5)
+    d = binding.to_device(w)
+    out = torch.full((2, 3), 123, dtype=torch.int32, device="cuda")
+    n = torch.full((2,), 77, dtype=torch.int32, device="cuda")
+    tiny = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(binding.SpecVerifyError):
+        binding.verify(**d, out_tokens=out, out_n_accepted=n, workspace=tiny)
+    torch.cuda.synchronize()
+    assert (out == 123).all() and (n == 77).all()
+
+
+def test_streams_and_graph_capture():
+    """The call is stream-ordered and capturable in a CUDA graph."""
+    w = W.make_workload("c1")
+    d = binding.to_device(w)
+    ref_t, ref_n = [t.clone() for t in binding.verify(**d)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        t2, n2 = binding.verify(**d)
+    torch.cuda.current_stream().wait_stream(s)
+    assert torch.equal(t2, ref_t) and torch.equal(n2, ref_n)
+    out_t = torch.empty_like(ref_t)
+    out_n = torch.empty_like(ref_n)
+    g = torch.cuda.CUDAGraph()
+    ws = binding.workspace_for(w.B, w.gamma, w.V, torch.float32, "cuda")
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        binding.verify(**d, out_tokens=out_t, out_n_accepted=out_n, workspace=ws)
+    for _ in range(3):
+        out_t.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out_t, ref_t) and torch.equal(out_n, ref_n)
