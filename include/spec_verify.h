@@ -133,6 +133,42 @@ sv_status spec_verify(const void* target_logits, const void* draft_logits, sv_dt
 /* Static description of a status code; never NULL. */
 const char* spec_verify_status_string(sv_status status);
 
+/*
+ * No-allocation variant.  The pages have no counterpart to this entry point;
+ * it exists for callers that must not allocate device memory themselves: code
+ * running inside another runtime's enqueue hook (an inference-engine plugin,
+ * for example) or under a fixed memory budget owned by someone else, where a
+ * cudaMalloc is forbidden or would synchronise the device in the middle of a
+ * decode step.
+ *
+ * Same arguments and results as spec_verify(), minus the workspace: the
+ * scratch lives in a fixed device array inside this library,
+ * SV_NOALLOC_SCRATCH_BYTES bytes on every GPU that loads the library, held
+ * until the process exits.  The caller still passes every input and output.
+ *
+ *  - Shapes whose workspace (spec_verify_workspace_size) exceeds
+ *    SV_NOALLOC_SCRATCH_BYTES are rejected with SV_ERR_WORKSPACE_TOO_SMALL
+ *    before anything is launched.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any stream
+ *    capture begins.
+ *  - The call allocates nothing: it clears the completion counters with
+ *    cudaMemsetAsync on `stream` and then launches the same kernels as
+ *    spec_verify().
+ *  - Every call shares the one array and leaves its contents behind, so calls
+ *    that overlap on the GPU (different streams without ordering, or several
+ *    host threads) race and give wrong results.  Order them.
+ */
+#define SV_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+sv_status spec_verify_noalloc(const void* target_logits, const void* draft_logits, sv_dtype dt,
+                              const int32_t* draft_tokens, const float* temperature,
+                              const float* u_accept, const float* u_resample,
+                              int32_t* out_tokens, int32_t* out_n_accepted,
+                              int B, int gamma, int V,
+                              double* out_log_norm, int32_t* out_row_status,
+                              struct CUstream_st* stream);
+
 #ifdef __cplusplus
 }
 #endif

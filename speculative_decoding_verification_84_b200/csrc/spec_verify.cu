@@ -33,6 +33,7 @@
 
 #include <cuda_runtime.h>
 #include <float.h>
+#include <mutex>
 #include <math.h>
 #include <stdint.h>
 
@@ -940,4 +941,66 @@ extern "C" const char* spec_verify_status_string(sv_status s)
     case SV_ERR_CUDA: return "CUDA launch or runtime error";
     }
     return "unknown status";
+}
+
+// ============================================================================= no-allocation variant
+//
+// For callers that cannot allocate device memory (see spec_verify_noalloc in the
+// header): the workspace is this fixed array, one per GPU for the life of the
+// process.  Host code must not pass the symbol itself to a kernel (on the host it
+// names a stand-in, not device memory); its device address is looked up once per
+// device below.
+
+static __device__ __align__(256) unsigned char sv_noalloc_scratch[SV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of sv_noalloc_scratch on the current device (first use per device
+// does the lookup).  Returns nullptr on a CUDA error.
+void* noalloc_scratch_address()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, sv_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" sv_status spec_verify_noalloc(const void* target_logits, const void* draft_logits, sv_dtype dt,
+                                         const int32_t* draft_tokens, const float* temperature,
+                                         const float* u_accept, const float* u_resample, int32_t* out_tokens,
+                                         int32_t* out_n_accepted, int B, int gamma, int V, double* out_log_norm,
+                                         int32_t* out_row_status, struct CUstream_st* stream)
+{
+    if (dt != SV_DTYPE_F32 && dt != SV_DTYPE_BF16) return SV_ERR_UNSUPPORTED_DTYPE;
+    Plan p;
+    if (!make_plan(B, gamma, V, dt, &p)) return SV_ERR_INVALID_ARG;
+    if (!target_logits || !draft_logits || !draft_tokens || !temperature || !u_accept || !u_resample ||
+        !out_tokens || !out_n_accepted)
+        return SV_ERR_INVALID_ARG;
+    if (!aligned(target_logits, 16) || !aligned(draft_logits, 16) || !aligned(draft_tokens, 4) ||
+        !aligned(temperature, 4) || !aligned(u_accept, 4) || !aligned(u_resample, 4) || !aligned(out_tokens, 4) ||
+        !aligned(out_n_accepted, 4) || !aligned(out_log_norm, 8) || !aligned(out_row_status, 4))
+        return SV_ERR_MISALIGNED;
+    if (p.total > SV_NOALLOC_SCRATCH_BYTES) return SV_ERR_WORKSPACE_TOO_SMALL;
+    unsigned char* ws = static_cast<unsigned char*>(noalloc_scratch_address());
+    if (!ws) return SV_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the completion counters must start at zero; the rest is overwritten before use
+    if (cudaMemsetAsync(ws, 0, p.off_seq, st) != cudaSuccess) return SV_ERR_CUDA;
+    const cudaError_t e =
+        dt == SV_DTYPE_BF16
+            ? launch<2>(p, target_logits, draft_logits, draft_tokens, temperature, u_accept, u_resample, out_tokens,
+                        out_n_accepted, out_log_norm, out_row_status, ws, st)
+            : launch<4>(p, target_logits, draft_logits, draft_tokens, temperature, u_accept, u_resample, out_tokens,
+                        out_n_accepted, out_log_norm, out_row_status, ws, st);
+    return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }
