@@ -184,7 +184,9 @@ def run_ours(args):
     wspace = torch.zeros(wsz, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     dt_code = binding._dt_code(tdt)
-    kernels_per_call = 2
+    kernels_per_call = binding.kernels_per_call(B, gamma, V, tdt)
+    kernel_name = "sv_stream (persistent, one launch per call)" if kernels_per_call == 1 else \
+        "sv_rowpass + sv_resample"
 
     def call(d):
         st = lib.spec_verify(d["target"].data_ptr(), d["draft"].data_ptr(), dt_code, d["draft_tokens"].data_ptr(),
@@ -295,7 +297,7 @@ def run_ours(args):
         "hbm_gbs": achieved, "pct_of_peak": 100.0 * achieved / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
-                     "kernel": "spec_verify call (sv_rowpass + sv_resample)",
+                     "kernel": kernel_name,
                      "algorithmic_bytes_per_launch": alg, "mean_launch_us": 1e3 * mean_call_ms,
                      "p10_us": 1e3 * float(np.percentile(per_call, 10)),
                      "p90_us": 1e3 * float(np.percentile(per_call, 90))},

@@ -83,14 +83,19 @@ typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
  * Bytes of device workspace spec_verify() needs for this shape (0 on a bad
  * shape).  The workspace is caller-owned device memory, 256-byte aligned.
  *
- * Its first 8*B bytes are completion counters that must be zero when a call
- * starts.  Zero the whole workspace once after allocating it (for example with
- * spec_verify_workspace_init); every call that runs to completion leaves the
- * counters at zero again, so one workspace serves any number of calls with the
- * same (B, gamma, V, dt).  Zero it again before reusing it for another shape.
- * Calls that share a workspace must be ordered (same stream, or events).
+ * Zero the whole workspace once after allocating it (for example with
+ * spec_verify_workspace_init).  It then serves any number of calls with the same
+ * (B, gamma, V, dt): every call that runs to completion leaves it ready for the
+ * next.  Zero it again before reusing it for another shape.  Calls that share a
+ * workspace must be ordered (same stream, or events).  The 8 bytes at offset 16
+ * are an error word: nonzero only if one of the kernel's bounded waits gave up
+ * (results of that call are then unreliable).
  */
 size_t spec_verify_workspace_size(int B, int gamma, int V, sv_dtype dt);
+
+/* Number of kernel launches one spec_verify() call of this shape enqueues
+ * (1 for the streaming kernel, 2 for the general path), or 0 on a bad shape. */
+int spec_verify_kernels_per_call(int B, int gamma, int V, sv_dtype dt);
 
 /* cudaMemsetAsync(workspace, 0, workspace_bytes, stream). */
 sv_status spec_verify_workspace_init(void* workspace, size_t workspace_bytes,
@@ -154,7 +159,8 @@ const char* spec_verify_status_string(sv_status status);
  *    capture begins.
  *  - The call allocates nothing: it clears the completion counters with
  *    cudaMemsetAsync on `stream` and then launches the same kernels as
- *    spec_verify().
+ *    spec_verify() (shapes served by the general two-kernel path also clear
+ *    their partial results afterwards, since the array serves every shape).
  *  - Every call shares the one array and leaves its contents behind, so calls
  *    that overlap on the GPU (different streams without ordering, or several
  *    host threads) race and give wrong results.  Order them.

@@ -20,7 +20,9 @@ SV_OK = 0
 SV_DTYPE_F32, SV_DTYPE_BF16 = 0, 1
 ROW_BAD_TOKEN, ROW_BAD_LOGITS, ROW_BAD_TEMPERATURE, ROW_RESIDUAL_ZERO = 1, 2, 4, 8
 EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_init",
-            "spec_verify_status_string")
+            "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc")
+# byte offset of the error word in a workspace (nonzero only if a bounded wait gave up)
+WORKSPACE_ERROR_OFFSET = 16
 
 _lib = None
 
@@ -48,6 +50,8 @@ def load_library(path: str = LIB_PATH):
     lib.spec_verify_workspace_init.restype = i32
     lib.spec_verify.argtypes = [vp, vp, i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, vp, vp, vp]
     lib.spec_verify.restype = i32
+    lib.spec_verify_kernels_per_call.argtypes = [i32, i32, i32, i32]
+    lib.spec_verify_kernels_per_call.restype = i32
     lib.spec_verify_status_string.argtypes = [i32]
     lib.spec_verify_status_string.restype = ctypes.c_char_p
     if path == LIB_PATH:
@@ -69,6 +73,15 @@ def _dt_code(dtype: torch.dtype) -> int:
 
 def workspace_size(B: int, gamma: int, V: int, dtype: torch.dtype) -> int:
     return int(load_library().spec_verify_workspace_size(B, gamma, V, _dt_code(dtype)))
+
+
+def kernels_per_call(B: int, gamma: int, V: int, dtype: torch.dtype) -> int:
+    return int(load_library().spec_verify_kernels_per_call(B, gamma, V, _dt_code(dtype)))
+
+
+def workspace_error(ws: torch.Tensor) -> int:
+    """The workspace's error word (0 unless a bounded device wait gave up)."""
+    return int(ws[WORKSPACE_ERROR_OFFSET:WORKSPACE_ERROR_OFFSET + 8].cpu().view(torch.int64).item())
 
 
 _ws_cache: Dict[Tuple, torch.Tensor] = {}

@@ -15,6 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "spec_verify.cu")
+DEPS = [os.path.join(HERE, "csrc", f) for f in ("sv_common.cuh", "sv_generic.cuh", "sv_stream.cuh")]
 HEADER = os.path.join(ROOT, "include", "spec_verify.h")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libspecverify.so")
@@ -32,7 +33,7 @@ def nvcc() -> str:
 
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(LIB_DIR, exist_ok=True)
-    newest = max(os.path.getmtime(SRC), os.path.getmtime(HEADER))
+    newest = max(os.path.getmtime(f) for f in [SRC, HEADER, *DEPS])
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"

@@ -97,16 +97,32 @@ def test_golden_worked_example_gpu():
         assert toks[i].tolist() == c["expect_tokens"], c["derivation"]
 
 
-def test_deterministic_and_workspace_reuse():
+@pytest.mark.parametrize("name", ["c2", "c3"])
+def test_deterministic_and_workspace_reuse(name):
     """Same inputs -> identical outputs over repeated calls on one workspace (the
-    completion counters reset themselves)."""
-    w = W.make_workload("c2")
+    counters and flags reset themselves); the workspace error word stays 0."""
+    w = W.make_workload(name)
     d = binding.to_device(w)
     first = [t.clone() for t in binding.verify(**d, return_log_norm=True)]
     for _ in range(5):
         again = binding.verify(**d, return_log_norm=True)
         for x, y in zip(first, again):
             assert torch.equal(x, y)
+    ws = binding.workspace_for(w.B, w.gamma, w.V, d["target"].dtype, "cuda")
+    assert binding.workspace_error(ws) == 0
+
+
+def test_generic_kernel_family():
+    """The general two-kernel family, forced on shapes the streaming kernel takes."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, SPEC_VERIFY_FORCE_GENERIC="1")
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, os.path.join(here, "generic_path_check.py")], env=env,
+                       capture_output=True, text=True, timeout=900)
+    print(r.stdout[-3000:], r.stderr[-3000:])
+    assert r.returncode == 0
 
 
 def test_host_errors_leave_outputs_untouched():

@@ -69,7 +69,7 @@ def test_noalloc_matches_spec_verify_two_calls(first, second):
 
 def test_noalloc_rejects_oversized_shape():
     f = _noalloc_fn()
-    B, gamma, V = 2048, 8, 151936                     # needs more than the built-in scratch
+    B, gamma, V = 8192, 8, 151936                     # needs more than the built-in scratch
     assert binding.workspace_size(B, gamma, V, torch.bfloat16) > NOALLOC_SCRATCH_BYTES
     p = ctypes.c_void_p(1 << 20)                      # never dereferenced: rejected on the host
     rc = f(p, p, 1, p, p, p, p, p, p, B, gamma, V, None, None, None)
