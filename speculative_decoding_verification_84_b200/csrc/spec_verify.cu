@@ -2,10 +2,11 @@
 // The operation is specified in include/spec_verify.h.  This file plans a call
 // (which kernel family, how the vocabulary is split, where everything lives in
 // the workspace) and launches it:
-//   * sv_stream (sv_stream.cuh): one persistent warp-specialised CTA per SM,
-//     bulk-copy pipeline, pass 1 and the residual pass in one launch.  Used when
-//     every row is 16-byte aligned (V * element size a multiple of 16) and at
-//     least 4 KB long.
+//   * sv_pass1 + sv_pass2 (sv_pass.cuh): two persistent kernels; pass 1 gives
+//     every warp one contiguous span of the row stream, pass 2 finishes the
+//     sequences and then sums and draws from the residual rows.  Used when every
+//     row is 16-byte aligned (V * element size a multiple of 16) and at least
+//     4 KB long.
 //   * sv_rowpass + sv_resample (sv_generic.cuh): any shape.
 // SPEC_VERIFY_FORCE_GENERIC=1 in the environment selects the second family for
 // every shape (both compute the same results; tests use it to cover both).
@@ -15,11 +16,12 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "sv_common.cuh"
 #include "sv_generic.cuh"
-#include "sv_stream.cuh"
+#include "sv_pass.cuh"
 
 namespace {
 
@@ -36,7 +38,8 @@ struct Plan {
     int B, gamma, V, R, esz;
     bool stream;
     int nc1, C1, nc2, C2;           // generic
-    int IB, nI1, nI2;               // stream
+    int nslot, NT2, nI2;            // stream
+    long long nq;                   // stream: 16-byte vectors per row
     long long rowbytes;
     size_t off_cnt, off_t1, off_t2, off_ready, off_seq, off_part, off_rsum, total;
 };
@@ -64,10 +67,7 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     p->esz = dt == SV_DTYPE_BF16 ? 2 : 4;
     p->rowbytes = (long long)V * p->esz;
     const long long rows = (long long)B * p->R;
-    p->stream = !force_generic() && (p->rowbytes % 16 == 0) && (p->rowbytes >= kMinItemBytes);
-    // the streaming kernel indexes its work list with 32-bit counters
-    if (p->stream && (long long)(B + 2 * kSmCount) * (rows / B) * (p->rowbytes / kMinItemBytes + 3) > (1LL << 30))
-        p->stream = false;
+    p->stream = !force_generic() && (p->rowbytes % 16 == 0) && (p->rowbytes >= kStreamMinRowBytes);
 
     // generic split: ~32 KB per CTA, but at least ~2 CTAs per SM in total
     long long nc1 = cdiv(p->rowbytes, kPass1ChunkBytes);
@@ -87,19 +87,16 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     p->C2 = (int)((cdiv(V, nc2) + 7) / 8 * 8);
     p->nc2 = (int)cdiv(V, p->C2);
 
-    // streaming split: items of IB bytes (residual items IB/2 per row), about four
-    // items per SM in total, between kMinItemBytes and kMaxItemBytes
-    long long ib = rows * p->rowbytes / (4LL * kSmCount);
-    if (ib < kMinItemBytes) ib = kMinItemBytes;
-    if (ib > kMaxItemBytes) ib = kMaxItemBytes;
-    if (ib > cdiv(p->rowbytes, 32) * 32) ib = cdiv(p->rowbytes, 32) * 32;
-    ib = ib / 32 * 32;
-    p->IB = (int)ib;
-    p->nI1 = (int)cdiv(p->rowbytes, ib);
-    p->nI2 = (int)cdiv(p->rowbytes, ib / 2);
+    // streaming split: pass-1 spans of at least kSpanMin vectors (so a row meets
+    // at most nslot of them), 16 KB pass-2 chunks, 512-byte tiles
+    p->nq = p->rowbytes / 16;
+    p->nslot = (int)cdiv(p->nq, kSpanMin) + 1;
+    p->nI2 = (int)cdiv(p->nq, kP2Chunk);
+    p->NT2 = (int)cdiv(p->nq, kTileVecs);
 
-    const long long nparts = rows * (p->stream ? (long long)p->nI1 : p->nc1);
-    const long long nrsum = p->stream ? (long long)B * p->nI2 * kGW : (long long)B * p->nc2;
+    // stream: one Partial per chunk; one float per tile (two per 8-byte slot)
+    const long long nparts = rows * (p->stream ? (long long)p->nslot : p->nc1);
+    const long long nrsum = p->stream ? cdiv((long long)B * p->NT2, 2) : (long long)B * p->nc2;
     size_t off = 0;
     p->off_cnt = off;
     off += 4 * sizeof(unsigned long long);
@@ -135,23 +132,22 @@ int device_sm_count()
     return cache[dev];
 }
 
-template <int ESZ>
-cudaError_t stream_smem_attr()
+// Resident CTAs per SM of a 256-thread kernel on the current device (cached per
+// kernel and device; 0 on a CUDA error).
+template <class K>
+int ctas_per_sm(K kernel, int slot)
 {
     static std::mutex mu;
-    static bool done[kMaxDevices] = {};
+    static int cache[4][kMaxDevices] = {};
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
     std::lock_guard<std::mutex> lock(mu);
-    if (!done[dev]) {
-        e = cudaFuncSetAttribute(sv_stream<ESZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kStages * kMaxItemBytes);
-        if (e != cudaSuccess) return e;
-        done[dev] = true;
+    if (!cache[slot][dev]) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kPassThreads, 0) != cudaSuccess || n < 1) n = 0;
+        cache[slot][dev] = n;
     }
-    return cudaSuccess;
+    return cache[slot][dev];
 }
 
 template <int ESZ>
@@ -177,26 +173,47 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
     t.R = p.R;
 
     if (p.stream) {
-        cudaError_t e = stream_smem_attr<ESZ>();
+        PassArgs g;
+        g.t = t;
+        g.part = reinterpret_cast<Partial*>(ws + p.off_part);
+        g.tsum = reinterpret_cast<float*>(ws + p.off_rsum);
+        g.u_resample = u_res;
+        g.ticket2 = reinterpret_cast<unsigned*>(ws + p.off_t2);
+        g.ready = reinterpret_cast<unsigned*>(ws + p.off_ready);
+        g.err = reinterpret_cast<unsigned long long*>(ws + p.off_cnt) + 2;
+        g.nq = p.nq;
+        g.NT2 = p.NT2;
+        g.nI2 = p.nI2;
+        g.B = p.B;
+        // as many CTAs as are resident at once; pass 1 splits the row stream into
+        // one span per warp, pass 2 has no more CTAs than chunks
+        const int c1 = ctas_per_sm(sv_pass1<ESZ>, ESZ == 2 ? 0 : 1);
+        const int c2 = ctas_per_sm(sv_pass2<ESZ>, ESZ == 2 ? 2 : 3);
+        if (c1 < 1 || c2 < 1) return cudaErrorInvalidConfiguration;
+        const long long sms = device_sm_count();
+        const long long NQ = (long long)p.B * p.R * p.nq;
+        long long grid1 = sms * c1;
+        g.S = std::max<long long>(kSpanMin, cdiv(NQ, grid1 * kWarps));
+        grid1 = std::min<long long>(grid1, cdiv(cdiv(NQ, g.S), kWarps));
+        const long long grid2 = std::min<long long>(sms * c2, std::max<long long>(p.B, (long long)p.B * p.nI2));
+        // a row meets at most this many spans: the partial slots per row
+        g.t.nc = (int)(cdiv(p.nq, g.S) + 1);
+        sv_pass1<ESZ><<<(unsigned)grid1, kPassThreads, 0, st>>>(g);
+        cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        StreamArgs a;
-        a.t = t;
-        a.t.nc = p.nI1;
-        a.pw = reinterpret_cast<unsigned long long*>(ws + p.off_part);
-        a.u_resample = u_res;
-        a.ready = reinterpret_cast<unsigned*>(ws + p.off_ready);
-        a.counters = reinterpret_cast<unsigned long long*>(ws + p.off_cnt);
-        a.rw = reinterpret_cast<unsigned long long*>(ws + p.off_rsum);
-        a.IB = p.IB;
-        a.nI1 = p.nI1;
-        a.nI2 = p.nI2;
-        a.per_step = p.R * p.nI1 + p.nI2;
-        const int grid = device_sm_count();
-        a.D = (int)cdiv((long long)grid * (kStages + 1), a.per_step) + 1;
-        a.n_items = (long long)(p.B + a.D) * a.per_step;
-        a.rowbytes = p.rowbytes;
-        sv_stream<ESZ><<<grid, kStreamThreads, (size_t)kStages * p.IB, st>>>(a);
-        return cudaGetLastError();
+        // pass 2 as a programmatic dependent launch: it may start while pass 1's
+        // last CTAs run and waits on the device for pass 1's completion
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid2);
+        cfg.blockDim = dim3(kPassThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, sv_pass2<ESZ>, g);
     }
 
     GenericArgs g;
@@ -236,7 +253,7 @@ extern "C" int spec_verify_kernels_per_call(int B, int gamma, int V, sv_dtype dt
 {
     Plan p;
     if (!make_plan(B, gamma, V, dt, &p)) return 0;
-    return p.stream ? 1 : 2;
+    return 2;
 }
 
 extern "C" sv_status spec_verify_workspace_init(void* workspace, size_t workspace_bytes,

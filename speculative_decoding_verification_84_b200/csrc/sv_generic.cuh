@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kThreads) sv_rowpass(GenericArgs g)
 {
     __shared__ float s_red[3 * kWarps];
     __shared__ int s_last;
+    __shared__ TailSmem s_tail;
     const TailArgs& a = g.t;
 
     const int c = blockIdx.x % g.nc1;
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(kThreads) sv_rowpass(GenericArgs g)
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    sequence_tail<ESZ, kThreads, BlockSync>(a, b, threadIdx.x, FloatPartials{a.part});
+    sequence_tail<ESZ, kThreads, BlockSync>(a, b, threadIdx.x, FloatPartials{a.part}, s_tail);
 }
 
 // Sum of the weights over [v0, v1) (valid in thread 0).
