@@ -38,10 +38,10 @@ struct Plan {
     int B, gamma, V, R, esz;
     bool stream;
     int nc1, C1, nc2, C2;           // generic
-    int nslot, NT2, nI2;            // stream
+    int nslot, NT2;                 // stream
     long long nq;                   // stream: 16-byte vectors per row
     long long rowbytes;
-    size_t off_cnt, off_t1, off_t2, off_ready, off_seq, off_part, off_rsum, total;
+    size_t off_cnt, off_t1, off_t2, off_ready, off_seq, off_gath, off_part, off_rsum, total;
 };
 
 __host__ inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -88,10 +88,9 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     p->nc2 = (int)cdiv(V, p->C2);
 
     // streaming split: pass-1 spans of at least kSpanMin vectors (so a row meets
-    // at most nslot of them), 16 KB pass-2 chunks, 512-byte tiles
+    // at most nslot of them), 512-byte tiles for the draw
     p->nq = p->rowbytes / 16;
     p->nslot = (int)cdiv(p->nq, kSpanMin) + 1;
-    p->nI2 = (int)cdiv(p->nq, kP2Chunk);
     p->NT2 = (int)cdiv(p->nq, kTileVecs);
 
     // stream: one Partial per chunk; one float per tile (two per 8-byte slot)
@@ -109,6 +108,8 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     off = align256(off);
     p->off_seq = off;
     off = align256(off + sizeof(SeqRec) * (size_t)B);
+    p->off_gath = off;
+    off = align256(off + (p->stream ? sizeof(float) * 2 * (size_t)gamma * B : 0));
     p->off_part = off;
     off = align256(off + sizeof(Partial) * (size_t)nparts);
     p->off_rsum = off;
@@ -150,6 +151,34 @@ int ctas_per_sm(K kernel, int slot)
     return cache[slot][dev];
 }
 
+// Clusters of cs CTAs of sv_pass2 that can be resident at once on the current
+// device (cached per cluster size and device; 0 on a CUDA error).
+template <int ESZ>
+int max_clusters(int cs)
+{
+    static std::mutex mu;
+    static int cache[kMaxCluster + 1][kMaxDevices] = {};
+    int dev = 0;
+    if (cs < 1 || cs > kMaxCluster || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[cs][dev]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(cs * device_sm_count()));
+        cfg.blockDim = dim3(kPassThreads);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, sv_pass2<ESZ>, &cfg) != cudaSuccess || n < 1) n = -1;
+        cache[cs][dev] = n;
+    }
+    return cache[cs][dev];
+}
+
 template <int ESZ>
 cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_t* tokens,
                    const float* temperature, const float* u_acc, const float* u_res, int32_t* out_tokens,
@@ -168,6 +197,7 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
     t.ticket = reinterpret_cast<unsigned*>(ws + p.off_t1);
     t.seq = reinterpret_cast<SeqRec*>(ws + p.off_seq);
     t.part = reinterpret_cast<const Partial*>(ws + p.off_part);
+    t.gath = nullptr;
     t.gamma = p.gamma;
     t.V = p.V;
     t.R = p.R;
@@ -176,43 +206,59 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
         PassArgs g;
         g.t = t;
         g.part = reinterpret_cast<Partial*>(ws + p.off_part);
+        g.gath = reinterpret_cast<float*>(ws + p.off_gath);
+        g.t.gath = g.gath;
         g.tsum = reinterpret_cast<float*>(ws + p.off_rsum);
         g.u_resample = u_res;
-        g.ticket2 = reinterpret_cast<unsigned*>(ws + p.off_t2);
-        g.ready = reinterpret_cast<unsigned*>(ws + p.off_ready);
-        g.err = reinterpret_cast<unsigned long long*>(ws + p.off_cnt) + 2;
         g.nq = p.nq;
         g.NT2 = p.NT2;
-        g.nI2 = p.nI2;
         g.B = p.B;
-        // as many CTAs as are resident at once; pass 1 splits the row stream into
-        // one span per warp, pass 2 has no more CTAs than chunks
+        // pass 1: as many CTAs as are resident at once, the row stream split into
+        // one span per warp
         const int c1 = ctas_per_sm(sv_pass1<ESZ>, ESZ == 2 ? 0 : 1);
-        const int c2 = ctas_per_sm(sv_pass2<ESZ>, ESZ == 2 ? 2 : 3);
-        if (c1 < 1 || c2 < 1) return cudaErrorInvalidConfiguration;
+        if (c1 < 1) return cudaErrorInvalidConfiguration;
         const long long sms = device_sm_count();
         const long long NQ = (long long)p.B * p.R * p.nq;
         long long grid1 = sms * c1;
         g.S = std::max<long long>(kSpanMin, cdiv(NQ, grid1 * kWarps));
         grid1 = std::min<long long>(grid1, cdiv(cdiv(NQ, g.S), kWarps));
-        const long long grid2 = std::min<long long>(sms * c2, std::max<long long>(p.B, (long long)p.B * p.nI2));
         // a row meets at most this many spans: the partial slots per row
         g.t.nc = (int)(cdiv(p.nq, g.S) + 1);
         sv_pass1<ESZ><<<(unsigned)grid1, kPassThreads, 0, st>>>(g);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        // pass 2 as a programmatic dependent launch: it may start while pass 1's
-        // last CTAs run and waits on the device for pass 1's completion
+
+        // pass 2: clusters of cs CTAs, one per sequence at a time; the largest
+        // cs (<= kMaxCluster) for which one wave of resident clusters covers the
+        // batch, else 1
+        int cs = 1, nclusters = 0;
+        for (int c = kMaxCluster; c >= 1; c >>= 1) {
+            const int n = max_clusters<ESZ>(c);
+            if (n < 1) continue;
+            if (c == 1 || (long long)n >= p.B) {
+                cs = c;
+                nclusters = n;
+                break;
+            }
+        }
+        if (nclusters < 1) return cudaErrorInvalidConfiguration;
+        const long long grid2 = (long long)cs * std::min<long long>(nclusters, p.B);
+        // a programmatic dependent launch: pass 2 may start while pass 1's last
+        // CTAs run, and waits on the device for pass 1's completion
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid2);
         cfg.blockDim = dim3(kPassThreads);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)cs;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         return cudaLaunchKernelEx(&cfg, sv_pass2<ESZ>, g);
     }
 

@@ -494,6 +494,7 @@ struct TailArgs {
     unsigned* ticket;
     SeqRec* seq;
     const Partial* part;
+    const float* gath;    // optional [B][2*gamma]: l_t[j][x_j] then l_d[j][x_j], gathered while streaming
     int gamma, V, R, nc;  // nc = partials per row
 };
 
@@ -541,10 +542,16 @@ __device__ void sequence_tail(const TailArgs& a, int b, int tid, const READ& rea
     double lt_j = 0.0, ld_j = 0.0, lu_j = 0.0;
     if (warp == 0 && lane < gamma && tval) {
         x_j = tok[lane];
+        if (a.gath) {  // the streaming pass stored them: no load that waits for x_j
+            lt_j = (double)__ldcg(a.gath + (size_t)b * 2 * gamma + lane);
+            ld_j = (double)__ldcg(a.gath + (size_t)b * 2 * gamma + gamma + lane);
+        }
         if (!greedy && x_j >= 0 && x_j < a.V) {
             const size_t V = (size_t)a.V;
-            lt_j = (double)load_logit<ESZ>(a.tgt, ((size_t)b * (gamma + 1) + lane) * V + x_j);
-            ld_j = (double)load_logit<ESZ>(a.dft, ((size_t)b * gamma + lane) * V + x_j);
+            if (!a.gath) {
+                lt_j = (double)load_logit<ESZ>(a.tgt, ((size_t)b * (gamma + 1) + lane) * V + x_j);
+                ld_j = (double)load_logit<ESZ>(a.dft, ((size_t)b * gamma + lane) * V + x_j);
+            }
             lu_j = log((double)a.u_accept[(size_t)b * gamma + lane]);
         }
     }

@@ -10,18 +10,23 @@
 //             few times) the warp reduces with shuffles and writes one Partial for
 //             that row segment.  A barrier per chunk would make every CTA wait for
 //             its slowest load; independent warps keep HBM busy.
-//   sv_pass2  first, CTA k finishes sequences b = k, k + grid, ...: fp64 combine
-//             of b's partials, gather, log-space accept scan [FlashSpec,
-//             Metodologia 1] (sequence_tail), then raises ready[b].  Then chunks
-//             (b, c), 2048 vectors of the row pair the extra token of b is drawn
-//             from (residual max(0, p_n - q_n), or p_gamma for the bonus)
-//             [Speculative Speculative Decoding, Metodologia 2], each warp
-//             turning 32 consecutive vectors (a tile) into one fp32 weight sum.
-//             A chunk waits (bounded) for ready[b]; the CTA that takes the last
-//             chunk of b draws the token by inverse CDF over b's tile sums.
-// Grids hold as many CTAs as are resident at once (pass 1: 4 per SM at 256
-// threads and at most 64 registers; pass 2: 2 per SM, so that the finish and the
-// draw run in registers), so every warp streams from start to end.  Pass 2 is
+//             The warp whose segment holds a row's draft token x_j also stores
+//             the logit l[x_j] for the accept test.
+//   sv_pass2  one thread-block cluster per sequence b (clusters loop over the
+//             sequences): rank 0 finishes b -- fp64 combine of its partials,
+//             log-space accept scan [FlashSpec, Metodologia 1] (sequence_tail) --
+//             and a cluster barrier (hardware, no polling) hands the outcome to
+//             the cluster through distributed shared memory.  The cluster's CTAs
+//             then split the row pair the extra token is drawn from (residual
+//             max(0, p_n - q_n), or p_gamma for the bonus) [Speculative
+//             Speculative Decoding, Metodologia 2], each warp turning 32
+//             consecutive vectors (a tile) into one fp32 weight sum; after a
+//             second cluster barrier rank 0 draws the token by inverse CDF over
+//             b's tile sums.
+// Pass 1's grid holds as many CTAs as are resident at once (4 per SM at 256
+// threads and at most 64 registers), so every warp streams from start to end.
+// Pass 2 runs 2 CTAs per SM (the finish and the draw run in registers), in
+// clusters of up to 8 sized so that one wave covers the batch when it can; it is
 // launched as a programmatic dependent of pass 1: its CTAs start as pass-1 CTAs
 // leave and wait (griddepcontrol.wait) for all of pass 1 before reading.
 #pragma once
@@ -29,12 +34,15 @@
 #include "sv_common.cuh"
 #include "sv_generic.cuh"
 
+#include <cooperative_groups.h>
+
 namespace sv {
+
+namespace cg = cooperative_groups;
 
 constexpr int kPassThreads = 256;                  // = kThreads: reduce_lse / reduce_amax apply
 constexpr int kP1Vec = 8;                          // 16-byte vectors per lane per pass-1 batch
-constexpr int kP2Vec = 8;                          // vectors per thread per row in a pass-2 chunk
-constexpr int kP2Chunk = kPassThreads * kP2Vec;    // 2048 vectors: 64 tiles
+constexpr int kMaxCluster = 8;                     // pass-2 cluster size limit (portable)
 constexpr int kTileVecs = 32;                      // vectors per tile (one per lane)
 constexpr int kStreamMinRowBytes = 4096;           // shorter rows take the generic path
 constexpr int kDrawQ = 16;                         // tile sums per lane per draw block
@@ -43,17 +51,14 @@ constexpr int kSpanMin = 512;                      // shortest pass-1 span (vect
 static_assert(kPassThreads == kThreads, "block reductions assume kThreads threads");
 
 struct PassArgs {
-    TailArgs t;              // t.nc = partial slots per row (stride and count)
+    TailArgs t;              // t.nc = partial slots per row (stride and count); t.gath = gath
     Partial* part;           // [B][R][t.nc]; the slots no span fills hold empty partials
+    float* gath;             // [B][2*gamma] the accept test's logits, written by pass 1
     float* tsum;             // [B][NT2] weight sum of each tile
     const float* u_resample;
-    unsigned* ticket2;       // [B] pass-2 chunks done
-    unsigned* ready;         // [B] 1 once b is finished (pass 2)
-    unsigned long long* err; // error word: bit 1 = a wait for ready[b] gave up
     long long nq;            // 16-byte vectors per row
     long long S;             // vectors per warp span (pass 1)
     int NT2;                 // tiles per row
-    int nI2;                 // pass-2 chunks per row
     int B;
 };
 
@@ -158,7 +163,19 @@ __device__ __forceinline__ void pass1_segment(const PassArgs& g, int b, int r, l
             const float os = __shfl_xor_sync(0xffffffffu, L.s, o);
             lse_merge(L, om, omk, os);
         }
-        if (lane == 0) *dst = Partial{L.m, L.mk, L.m == -INFINITY ? 0.f : L.s, 0};
+        if (lane == 0) {
+            *dst = Partial{L.m, L.mk, L.m == -INFINITY ? 0.f : L.s, 0};
+            // the accept test's logit l[x_j] of this row, if the segment holds it
+            // (target rows j < gamma and draft rows j; the bonus row has no token)
+            if (r != a.gamma) {
+                const int j = r < a.gamma ? r : r - a.gamma - 1;
+                const int x = __ldg(a.tokens + (size_t)b * a.gamma + j);
+                const long long e = (long long)x - q0 * VEC;
+                if (x >= 0 && x < a.V && e >= 0 && e < (long long)n * VEC)
+                    g.gath[(size_t)b * 2 * a.gamma + (r < a.gamma ? j : a.gamma + j)] =
+                        load_logit<ESZ>(p, (size_t)e);
+            }
+        }
     }
 }
 
@@ -378,116 +395,84 @@ __device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& 
     }
 }
 
-__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p)
+// Weight sums of tiles [k0, k1) of the row pair, one per warp-tile: warp w takes
+// tiles k0 + 8*(4j + u) + w (u < 4), lane l vector 32k + l, so each lane has 4
+// (or 8, with the draft row) loads in flight.  Vectors past the row read as -inf
+// target logits, whose weight is 0.
+template <int ESZ, bool PONLY>
+__device__ void tile_range(const PassArgs& g, const SeqRec& rec, const uint4* tv, const uint4* dv, float* dst,
+                           int k0, int k1)
 {
-    unsigned v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Thread 0 waits for ready[b] (relaxed loads with back-off, one fence after);
-// false after kWaitLimitNs or once the error word is set.
-__device__ bool wait_ready(const PassArgs& g, int b)
-{
-    if (ld_relaxed_u32(g.ready + b) != 1u) {
-        const unsigned long long t0 = global_ns();
-        unsigned sleep = 64;
-        for (unsigned it = 0;; ++it) {
-            __nanosleep(sleep);
-            if (sleep < 1024) sleep *= 2;
-            if (ld_relaxed_u32(g.ready + b) == 1u) break;
-            if ((it & 3u) == 3u && (it > (1u << 24) || ld_relaxed_u64(g.err) != 0ull || global_ns() - t0 > kWaitLimitNs))
-                return false;
+    constexpr int VEC = 16 / ESZ;
+    constexpr int U = 4;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int kb = k0 + warp; kb < k1; kb += U * kWarps) {
+        uint4 vt[U], vd[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = kb + u * kWarps;
+            const long long q = (long long)k * kTileVecs + lane;
+            const bool ok = k < k1 && q < g.nq;
+            vt[u] = ok ? ld_stream(tv + q) : neg_inf_vec<ESZ>();
+            if (!PONLY) vd[u] = ok ? ld_stream(dv + q) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float xt[VEC], xd[VEC];
+            float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            unpack<ESZ>(vt[u], xt);
+            if (!PONLY) unpack<ESZ>(vd[u], xd);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) w[e] = weight_of(rec, PONLY, xt[e], PONLY ? 0.f : xd[e]);
+            float sum = tree8(w);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            const int k = kb + u * kWarps;
+            if (lane == 0 && k < k1) dst[k] = sum;
         }
     }
-    __threadfence();
-    return true;
 }
 
 template <int ESZ>
-__device__ __noinline__ void pass2_finish(const PassArgs& g, int b, TailSmem& ts)
+__device__ __noinline__ void pass2_finish(const PassArgs& g, int b, TailSmem& ts, SeqRec* rec_out)
 {
     const TailArgs& a = g.t;
     sequence_tail<ESZ, kPassThreads, BlockSync>(a, b, threadIdx.x, FloatPartials{a.part}, ts);
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicExch(g.ready + b, 1u);
-    }
+    if (threadIdx.x == 0) *rec_out = a.seq[b];  // written by this CTA's thread 0
 }
 
 template <int ESZ>
 __global__ void __launch_bounds__(kPassThreads, 2) sv_pass2(PassArgs g)
 {
-    constexpr int VEC = 16 / ESZ;
     __shared__ TailSmem s_tail;
-    __shared__ int s_last, s_ok;
+    __shared__ SeqRec s_rec;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank(), cs = (int)cluster.num_blocks();
+    const int cid = blockIdx.x / cs, nclusters = gridDim.x / cs;
     const TailArgs& t = g.t;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // wait until pass 1 has completed and its writes are visible (a no-op when
     // this launch did not overlap pass 1)
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    // finish this CTA's sequences
-    for (int b = blockIdx.x; b < g.B; b += gridDim.x) pass2_finish<ESZ>(g, b, s_tail);
 
-    const long long n_chunks = (long long)g.B * g.nI2;
-    for (long long ci = blockIdx.x; ci < n_chunks; ci += gridDim.x) {
-        const int b = (int)(ci / g.nI2);
-        const int c = (int)(ci - (long long)b * g.nI2);
-        if (tid == 0) {
-            s_ok = wait_ready(g, b) ? 1 : 0;
-            if (!s_ok) atomicOr(g.err, 1ull);
-        }
-        __syncthreads();
-        SeqRec rec;
-        rec.mode = kModeNone;
-        if (s_ok) rec = load_seqrec_cg(t.seq + b);
+    for (int b = cid; b < g.B; b += nclusters) {
+        if (rank == 0) pass2_finish<ESZ>(g, b, s_tail, &s_rec);
+        cluster.sync();  // rank 0's outcome (shared and global memory) is visible to the cluster
+        const SeqRec rec = *cluster.map_shared_rank(&s_rec, 0);
         if (rec.mode != kModeNone) {
-            const bool p_only = (rec.mode == kModeBonus);
+            const bool bonus = (rec.mode == kModeBonus);
             const uint4* tv = reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, rec.n));
-            const uint4* dv = p_only ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
-            const long long q0 = (long long)c * kP2Chunk;
-            uint4 vt[kP2Vec], vd[kP2Vec];
-#pragma unroll
-            for (int u = 0; u < kP2Vec; ++u) {
-                const long long q = q0 + u * kPassThreads + tid;
-                const bool ok = q < g.nq;
-                vt[u] = ok ? ld_stream(tv + q) : neg_inf_vec<ESZ>();  // -inf: weight 0
-                vd[u] = (ok && !p_only) ? ld_stream(dv + q) : make_uint4(0u, 0u, 0u, 0u);
-            }
+            const uint4* dv = bonus ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
             float* dst = g.tsum + (size_t)b * g.NT2;
-#pragma unroll
-            for (int u = 0; u < kP2Vec; ++u) {
-                float xt[VEC], xd[VEC];
-                float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                unpack<ESZ>(vt[u], xt);
-                unpack<ESZ>(vd[u], xd);
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) w[e] = weight_of(rec, p_only, xt[e], p_only ? 0.f : xd[e]);
-                float s = tree8(w);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                // warp `warp` covered vectors q0 + u*256 + 32*warp + [0, 32): one tile
-                const long long k = (q0 + u * kPassThreads) / kTileVecs + warp;
-                if (lane == 0 && k < g.NT2) dst[k] = s;
-            }
+            // this CTA's share of the tiles
+            const int per = (g.NT2 + cs - 1) / cs;
+            const int k0 = rank * per, k1 = min(g.NT2, k0 + per);
+            if (bonus) tile_range<ESZ, true>(g, rec, tv, tv, dst, k0, k1);
+            else tile_range<ESZ, false>(g, rec, tv, dv, dst, k0, k1);
         }
-        __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            s_last = atomicAdd(&g.ticket2[b], 1u) == (unsigned)(g.nI2 - 1);
-        }
-        __syncthreads();
-        if (s_last) {
-            // every chunk of b has passed its wait: ready for the next call
-            if (rec.mode != kModeNone) pass2_draw<ESZ>(g, b, rec);
-            if (tid == 0) {
-                g.ticket2[b] = 0u;
-                g.ready[b] = 0u;
-            }
-        }
-        __syncthreads();  // s_last and s_ok are rewritten by the next chunk
+        cluster.sync();  // every tile sum of b is visible to rank 0
+        if (rank == 0 && rec.mode != kModeNone) pass2_draw<ESZ>(g, b, rec);
     }
 }
 
