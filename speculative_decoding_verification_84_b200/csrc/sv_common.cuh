@@ -506,6 +506,7 @@ struct TailSmem {
     int arg[kMaxRows];
     int bad[kMaxRows];
     int status, n;
+    SeqRec rec;  // the draw record, also stored to seq[b]
 };
 
 // Finish sequence b once every partial of its rows is written: combine the
@@ -528,11 +529,12 @@ __device__ void sequence_tail(const TailArgs& a, int b, int tid, const READ& rea
 
     const int lane = tid & 31, warp = tid >> 5;
     const int gamma = a.gamma, R = a.R, nc = a.nc;
+    constexpr int kTailBatch = 8;
+    const size_t pbase = (size_t)b * R * nc;
     const float T = a.temperature[b];
     const bool greedy = (T == 0.f);
     const bool tval = temperature_ok(T);
     const int rows_used = !tval ? 0 : (greedy ? gamma + 1 : R);
-    const size_t pbase = (size_t)b * R * nc;
     const int32_t* tok = a.tokens + (size_t)b * gamma;
     float khi_t = 0.f, klo_t = 0.f;
     if (tval && !greedy) split_k(T, &khi_t, &klo_t);
@@ -559,7 +561,6 @@ __device__ void sequence_tail(const TailArgs& a, int b, int tid, const READ& rea
     // One thread per row: fold the row's partials in order.  Loads go out in
     // batches of kTailBatch before any arithmetic, so a batch costs one memory
     // latency.  Softmax rows merge (mk, s) exactly in fp64 (power-of-two scaling).
-    constexpr int kTailBatch = 8;
     for (int r = tid; r < rows_used; r += NT) {
         const size_t rbase = pbase + (size_t)r * nc;
         Amax A{-INFINITY, 0x7fffffff, 0};
@@ -670,6 +671,7 @@ __device__ void sequence_tail(const TailArgs& a, int b, int tid, const READ& rea
             }
         }
         a.seq[b] = rec;
+        sm.rec = rec;
         a.ticket[b] = 0u;  // every contribution has arrived: ready for the next call
     }
 }

@@ -43,6 +43,7 @@ namespace cg = cooperative_groups;
 constexpr int kPassThreads = 256;                  // = kThreads: reduce_lse / reduce_amax apply
 constexpr int kP1Vec = 8;                          // 16-byte vectors per lane per pass-1 batch
 constexpr int kMaxCluster = 8;                     // pass-2 cluster size limit (portable)
+constexpr int kTileSmem = 4096;                    // tile sums kept in rank 0's shared memory up to this many
 constexpr int kTileVecs = 32;                      // vectors per tile (one per lane)
 constexpr int kStreamMinRowBytes = 4096;           // shorter rows take the generic path
 constexpr int kDrawQ = 16;                         // tile sums per lane per draw block
@@ -214,13 +215,15 @@ struct TileBlock {
     double incl;  // inclusive prefix of ls over lanes
 };
 
-__device__ __forceinline__ void load_tile_block(TileBlock& tb, const float* w, int n, int s0)
+// w is either this CTA's shared memory (smem) or global memory written by other
+// CTAs of the cluster (read at L2).
+__device__ __forceinline__ void load_tile_block(TileBlock& tb, const float* w, int n, int s0, bool smem)
 {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int q = 0; q < kDrawQ; ++q) {
         const int idx = s0 + lane * kDrawQ + q;
-        tb.v[q] = idx < n ? __ldcg(w + idx) : 0.f;
+        tb.v[q] = idx < n ? (smem ? w[idx] : __ldcg(w + idx)) : 0.f;
     }
     double s = 0.0;
 #pragma unroll
@@ -266,12 +269,12 @@ __device__ __forceinline__ int walk_tile_block(const TileBlock& tb, int s0, doub
 }
 
 // Sum of all tile sums of a sequence, in the block order walk_tile_block uses.
-__device__ double tiles_total(const float* w, int n)
+__device__ double tiles_total(const float* w, int n, bool smem)
 {
     double carry = 0.0;
     for (int s0 = 0; s0 < n; s0 += 32 * kDrawQ) {
         TileBlock tb;
-        load_tile_block(tb, w, n, s0);
+        load_tile_block(tb, w, n, s0, smem);
         carry += __shfl_sync(0xffffffffu, tb.incl, 31);
     }
     return carry;
@@ -352,19 +355,17 @@ __device__ void tile_sums_strided(const PassArgs& g, const SeqRec& rec, bool p_o
 // smallest token k with C_k > u * S over b's tile sums; a vanished residual
 // (S = 0) falls back to p_n, whose tile sums the CTA computes first.
 template <int ESZ>
-__device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& rec)
+__device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& rec, float* ws, bool smem)
 {
     __shared__ double s_S;
     const TailArgs& t = g.t;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float* ws = g.tsum + (size_t)b * g.NT2;
     const int n = g.NT2;
     const bool bonus = (rec.mode == kModeBonus);
     const uint4* tv = reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, rec.n));
     const uint4* dv = bonus ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
-    __threadfence();  // the other chunks' tile sums, published before their tickets
     if (warp == 0) {
-        const double S = tiles_total(ws, n);
+        const double S = tiles_total(ws, n, smem);
         if (lane == 0) s_S = S;
     }
     __syncthreads();
@@ -378,13 +379,13 @@ __device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& 
         __syncthreads();
     }
     if (warp != 0) return;
-    const double S = flag ? tiles_total(ws, n) : s_S;
+    const double S = flag ? tiles_total(ws, n, smem) : s_S;
     const double target = (double)__ldg(g.u_resample + b) * S;
     int ts = -1;
     double base = 0.0, carry = 0.0;
     for (int s0 = 0; s0 < n && ts < 0; s0 += 32 * kDrawQ) {
         TileBlock tb;
-        load_tile_block(tb, ws, n, s0);
+        load_tile_block(tb, ws, n, s0, smem);
         ts = walk_tile_block(tb, s0, carry, target, &base);
         carry += __shfl_sync(0xffffffffu, tb.incl, 31);
     }
@@ -439,7 +440,7 @@ __device__ __noinline__ void pass2_finish(const PassArgs& g, int b, TailSmem& ts
     const TailArgs& a = g.t;
     sequence_tail<ESZ, kPassThreads, BlockSync>(a, b, threadIdx.x, FloatPartials{a.part}, ts);
     __syncthreads();
-    if (threadIdx.x == 0) *rec_out = a.seq[b];  // written by this CTA's thread 0
+    if (threadIdx.x == 0) *rec_out = ts.rec;
 }
 
 template <int ESZ>
@@ -447,10 +448,13 @@ __global__ void __launch_bounds__(kPassThreads, 2) sv_pass2(PassArgs g)
 {
     __shared__ TailSmem s_tail;
     __shared__ SeqRec s_rec;
+    __shared__ float s_tiles[kTileSmem];  // rank 0: b's tile sums, written by the whole cluster
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank(), cs = (int)cluster.num_blocks();
     const int cid = blockIdx.x / cs, nclusters = gridDim.x / cs;
     const TailArgs& t = g.t;
+    const bool tiles_in_smem = g.NT2 <= kTileSmem;
+    float* tiles0 = cluster.map_shared_rank(s_tiles, 0);  // rank 0's buffer, from any rank
 
     // wait until pass 1 has completed and its writes are visible (a no-op when
     // this launch did not overlap pass 1)
@@ -458,13 +462,13 @@ __global__ void __launch_bounds__(kPassThreads, 2) sv_pass2(PassArgs g)
 
     for (int b = cid; b < g.B; b += nclusters) {
         if (rank == 0) pass2_finish<ESZ>(g, b, s_tail, &s_rec);
-        cluster.sync();  // rank 0's outcome (shared and global memory) is visible to the cluster
+        cluster.sync();  // rank 0's outcome is visible to the cluster
         const SeqRec rec = *cluster.map_shared_rank(&s_rec, 0);
+        float* dst = tiles_in_smem ? tiles0 : g.tsum + (size_t)b * g.NT2;
         if (rec.mode != kModeNone) {
             const bool bonus = (rec.mode == kModeBonus);
             const uint4* tv = reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, rec.n));
             const uint4* dv = bonus ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
-            float* dst = g.tsum + (size_t)b * g.NT2;
             // this CTA's share of the tiles
             const int per = (g.NT2 + cs - 1) / cs;
             const int k0 = rank * per, k1 = min(g.NT2, k0 + per);
@@ -472,7 +476,9 @@ __global__ void __launch_bounds__(kPassThreads, 2) sv_pass2(PassArgs g)
             else tile_range<ESZ, false>(g, rec, tv, dv, dst, k0, k1);
         }
         cluster.sync();  // every tile sum of b is visible to rank 0
-        if (rank == 0 && rec.mode != kModeNone) pass2_draw<ESZ>(g, b, rec);
+        if (rank == 0 && rec.mode != kModeNone) pass2_draw<ESZ>(g, b, rec, tiles_in_smem ? s_tiles : dst, tiles_in_smem);
+        // rank 0's s_rec and s_tiles are rewritten for the next sequence only
+        // after the next iteration's finish, which the other ranks wait for
     }
 }
 
