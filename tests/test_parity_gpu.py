@@ -45,6 +45,15 @@ RAGGED = [
     (1, 4, 32003, "f32"), (9, 2, 8195, "f32"), (40, 2, 257, "bf16"),
 ]
 
+# 16-byte-aligned rows of at least 4 KB: the streaming kernels.  Short rows (one
+# pass-1 span covers several), gamma = 32 (65 rows per sequence), a ragged last
+# tile, draws over more than one block of tile sums, and rows whose tile sums do
+# not fit in shared memory (more than 4096 tiles).
+ALIGNED = [
+    (5, 3, 2056, "bf16"), (2, 32, 1032, "f32"), (7, 4, 40008, "bf16"), (11, 6, 12344, "f32"),
+    (1, 2, 250000, "f32"), (3, 1, 600000, "f32"), (90, 2, 4096, "bf16"),
+]
+
 
 @pytest.mark.parametrize("B,gamma,V,dt", RAGGED)
 def test_ragged_shapes(B, gamma, V, dt):
@@ -56,10 +65,23 @@ def test_ragged_shapes(B, gamma, V, dt):
     parity.assert_parity(st)
 
 
-def test_edge_cases():
-    """NaN / +inf / all -inf rows, out-of-range tokens, invalid temperatures, masked vocab."""
+@pytest.mark.parametrize("B,gamma,V,dt", ALIGNED)
+def test_aligned_shapes(B, gamma, V, dt):
+    """Shapes that take the streaming kernels, mixed T incl. greedy."""
+    assert (V * (2 if dt == "bf16" else 4)) % 16 == 0
+    T = np.array([0.0, 0.4, 1.0, 1.7, 1e-3][: 5] * ((B + 4) // 5), np.float32)[:B]
+    w = W.make_random(B, gamma, V, dt, seed=2000 + V + 7 * B + gamma, T=T)
+    st = parity.compare(parity.run_gpu(w), oracle.verify_workload(w))
+    _report(f"{B}x{gamma}x{V}-{dt}", st)
+    parity.assert_parity(st)
+
+
+@pytest.mark.parametrize("V", [300, 4096])
+def test_edge_cases(V):
+    """NaN / +inf / all -inf rows, out-of-range tokens, invalid temperatures, masked vocab
+    (V = 300: the general kernels; V = 4096 f32, 16 KB rows: the streaming kernels)."""
     rng = np.random.default_rng(9)
-    B, gamma, V = 14, 3, 300
+    B, gamma = 14, 3
     tgt = (rng.standard_normal((B, gamma + 1, V)) * 2).astype(np.float32)
     dft = (tgt[:, :gamma] + rng.standard_normal((B, gamma, V))).astype(np.float32)
     toks = rng.integers(0, V, (B, gamma)).astype(np.int32)
@@ -78,12 +100,12 @@ def test_edge_cases():
     tgt[11, 0, :] = 1.0                        # all-tie greedy row: index 0 wins
     toks[11, 0] = 0
     tgt[12, 0, :] = -np.inf                    # all -inf row
-    w = W.Workload("edges", "f32", tgt, dft, toks, T, W.draw_uniforms(rng, (B, gamma)),
+    w = W.Workload(f"edges-{V}", "f32", tgt, dft, toks, T, W.draw_uniforms(rng, (B, gamma)),
                    W.draw_uniforms(rng, (B,)))
     ref = oracle.verify_workload(w)
     assert ref.row_status[:9].tolist() == [2, 2, 2, 1, 1, 4, 4, 4, 4]
     st = parity.compare(parity.run_gpu(w), ref)
-    _report("edges", st)
+    _report(f"edges-{V}", st)
     parity.assert_parity(st)
 
 
