@@ -109,6 +109,21 @@ def dist_env():
     return ws, rank, local
 
 
+def job_value(local_ms, world, per_rank_units, pg=None, device=None):
+    """Whole-job throughput (units per second) and the job's time in ms.
+
+    Every rank processed its own per_rank_units; the job took as long as its
+    slowest rank, so the time is the max over ranks (an all-reduce over pg when
+    there is more than one rank)."""
+    total_ms = float(local_ms)
+    if pg is not None:
+        import torch
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    return world * per_rank_units / (total_ms / 1e3), total_ms
+
+
 def oracle_time(w, min_seconds, n_threads=0):
     """Time the oracle on the batch, repeated until min_seconds of CPU work; seq-steps/s."""
     import oracle
@@ -219,13 +234,8 @@ def run_ours(args):
     barrier()
     clocks = sampler.stop()
     per_call = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[args.steps])
-    if pg is not None:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    value, total_ms = job_value(ev[0].elapsed_time(ev[args.steps]), ws, B * args.steps, pg, dev)
     ms_per_step = total_ms / args.steps
-    value = ws * B * args.steps / (total_ms / 1e3)
 
     alg = algorithmic_bytes(B, gamma, V, esz)
     mean_call_ms = float(np.mean(per_call))
@@ -262,12 +272,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if pg is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = ws * B * e2e_steps / (e2e_ms / 1e3)
+    e2e_value, _ = job_value(e0.elapsed_time(e1), ws, B * e2e_steps, pg, dev)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

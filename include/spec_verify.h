@@ -88,13 +88,13 @@ typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
  * (B, gamma, V, dt): every call that runs to completion leaves it ready for the
  * next.  Zero it again before reusing it for another shape.  Calls that share a
  * workspace must be ordered (same stream, or events).  The 8 bytes at offset 16
- * are an error word: nonzero only if one of the kernel's bounded waits gave up
- * (results of that call are then unreliable).
+ * are reserved as an error word for kernels that wait on one another; the
+ * kernels of this version never do, so it stays zero.
  */
 size_t spec_verify_workspace_size(int B, int gamma, int V, sv_dtype dt);
 
-/* Number of kernel launches one spec_verify() call of this shape enqueues
- * (1 for the streaming kernel, 2 for the general path), or 0 on a bad shape. */
+/* Number of kernel launches one spec_verify() call of this shape enqueues (2
+ * for either kernel family), or 0 on a bad shape. */
 int spec_verify_kernels_per_call(int B, int gamma, int V, sv_dtype dt);
 
 /* cudaMemsetAsync(workspace, 0, workspace_bytes, stream). */
@@ -159,8 +159,7 @@ const char* spec_verify_status_string(sv_status status);
  *    capture begins.
  *  - The call allocates nothing: it clears the completion counters with
  *    cudaMemsetAsync on `stream` and then launches the same kernels as
- *    spec_verify() (shapes served by the general two-kernel path also clear
- *    their partial results afterwards, since the array serves every shape).
+ *    spec_verify().
  *  - Every call shares the one array and leaves its contents behind, so calls
  *    that overlap on the GPU (different streams without ordering, or several
  *    host threads) race and give wrong results.  Order them.

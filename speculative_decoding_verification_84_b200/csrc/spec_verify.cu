@@ -404,20 +404,14 @@ extern "C" sv_status spec_verify_noalloc(const void* target_logits, const void* 
     unsigned char* ws = static_cast<unsigned char*>(noalloc_scratch_address());
     if (!ws) return SV_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
-    // counters that must start at zero (claim, exit, error; the general path's
-    // tickets); the epoch word at offset 24 is kept, so tags never repeat
-    if (cudaMemsetAsync(ws, 0, 24, st) != cudaSuccess) return SV_ERR_CUDA;
-    if (cudaMemsetAsync(ws + 32, 0, p.off_seq - 32, st) != cudaSuccess) return SV_ERR_CUDA;
+    // what must start at zero: the error word and the general path's tickets
+    // (every call leaves them zero, but the array is shared by every shape)
+    if (cudaMemsetAsync(ws, 0, p.off_seq, st) != cudaSuccess) return SV_ERR_CUDA;
     const cudaError_t e =
         dt == SV_DTYPE_BF16
             ? launch<2>(p, target_logits, draft_logits, draft_tokens, temperature, u_accept, u_resample, out_tokens,
                         out_n_accepted, out_log_norm, out_row_status, ws, st)
             : launch<4>(p, target_logits, draft_logits, draft_tokens, temperature, u_accept, u_resample, out_tokens,
                         out_n_accepted, out_log_norm, out_row_status, ws, st);
-    if (e != cudaSuccess) return SV_ERR_CUDA;
-    // the array serves every shape: do not leave the general path's partials where
-    // a later streaming call of another shape looks for its tagged words
-    if (!p.stream && cudaMemsetAsync(ws + p.off_part, 0, p.total - p.off_part, st) != cudaSuccess)
-        return SV_ERR_CUDA;
-    return SV_OK;
+    return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }
