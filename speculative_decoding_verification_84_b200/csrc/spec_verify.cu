@@ -41,7 +41,7 @@ struct Plan {
     int nslot, NT2;                 // stream
     long long nq;                   // stream: 16-byte vectors per row
     long long rowbytes;
-    size_t off_cnt, off_t1, off_t2, off_ready, off_seq, off_gath, off_part, off_rsum, total;
+    size_t off_cnt, off_t1, off_t2, off_seq, off_gath, off_part, off_rsum, total;
 };
 
 __host__ inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -93,7 +93,7 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     p->nslot = (int)cdiv(p->nq, kSpanMin) + 1;
     p->NT2 = (int)cdiv(p->nq, kTileVecs);
 
-    // stream: one Partial per chunk; one float per tile (two per 8-byte slot)
+    // stream: one Partial per (row, span) slot; one float per tile (two per 8-byte slot)
     const long long nparts = rows * (p->stream ? (long long)p->nslot : p->nc1);
     const long long nrsum = p->stream ? cdiv((long long)B * p->NT2, 2) : (long long)B * p->nc2;
     size_t off = 0;
@@ -102,8 +102,6 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     p->off_t1 = off;
     off += sizeof(unsigned) * (size_t)B;
     p->off_t2 = off;
-    off += sizeof(unsigned) * (size_t)B;
-    p->off_ready = off;
     off += sizeof(unsigned) * (size_t)B;
     off = align256(off);
     p->off_seq = off;

@@ -11,7 +11,7 @@
 //                [Speculative Speculative Decoding, Metodologia 2: outcome =
 //                accepted count + extra token; residual distribution.]
 // Used when rows are not 16-byte aligned or are too short for the streaming
-// kernel in sv_stream.cuh.
+// kernels in sv_pass.cuh.
 #pragma once
 
 #include "sv_common.cuh"
