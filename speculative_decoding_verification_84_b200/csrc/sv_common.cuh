@@ -52,16 +52,9 @@ struct __align__(16) SeqRec {
     float k_lo;
 };
 
-// Barrier policies: the whole CTA, or only the compute warps of a
-// warp-specialised CTA (named barrier 1, kThreads threads).
+// Barrier policy of sequence_tail's callers: the whole CTA.
 struct BlockSync {
     static __device__ __forceinline__ void sync() { __syncthreads(); }
-};
-struct ConsumerSync {
-    static __device__ __forceinline__ void sync() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
-};
-struct WarpSync {
-    static __device__ __forceinline__ void sync() { __syncwarp(); }
 };
 
 // ----------------------------------------------------------------------------- loads and math
@@ -407,76 +400,14 @@ __device__ __forceinline__ float weight_of(const SeqRec& s, bool p_only, float l
 
 // ----------------------------------------------------------------------------- sequence tail
 
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p)
-{
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v)
-{
-    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long global_ns()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Longest a wait on another warp's result may take before it is declared lost.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
-
-// Readers of one (row, chunk) partial.  raw(i) issues the loads; value(raw, i,
-// khi, greedy) turns them into (m, mk, s, idx-bits).  The split lets a batch of
+// Reader of one (row, chunk) partial.  raw(i) issues the load; value(raw, i,
+// khi, greedy) turns it into (m, mk, s, idx-bits).  The split lets a batch of
 // loads be in flight before any of them is used.
 struct FloatPartials {  // Partial structs, published by a fenced ticket
     const Partial* p;
     using Raw = float4;
     __device__ __forceinline__ float4 raw(size_t i) const { return __ldcg(reinterpret_cast<const float4*>(p) + i); }
     __device__ __forceinline__ float4 value(const float4& r, size_t, float, bool) const { return r; }
-};
-
-// Two self-validating 64-bit words per partial, (value | tag << 32): word 0 holds
-// the max logit, word 1 the sum (softmax rows) or first index | NaN flag << 31
-// (greedy rows).  The integer offset is recomputed as ceil(m * k_hi), exactly as
-// its writer formed it.  A word that does not carry the tag yet is read again
-// until it does; after kWaitLimitNs (or once *err is non-zero) the partial reads
-// as NaN, which marks its row bad, and bit `err_bit` is set in *err.
-struct TaggedPartials {
-    const unsigned long long* w;
-    unsigned tag;
-    unsigned long long* err;
-    unsigned err_bit;
-    using Raw = ulonglong2;
-    __device__ __forceinline__ ulonglong2 raw(size_t i) const
-    {
-        return make_ulonglong2(ld_relaxed_u64(w + 2 * i), ld_relaxed_u64(w + 2 * i + 1));
-    }
-    __device__ float4 value(ulonglong2 r, size_t i, float khi, bool greedy) const
-    {
-        if ((unsigned)(r.x >> 32) != tag || (unsigned)(r.y >> 32) != tag) {
-            const unsigned long long t0 = global_ns();
-            for (unsigned it = 0;; ++it) {
-                __nanosleep(64);
-                r = raw(i);
-                if ((unsigned)(r.x >> 32) == tag && (unsigned)(r.y >> 32) == tag) break;
-                if (it > (1u << 26) || ld_relaxed_u64(err) != 0ull || global_ns() - t0 > kWaitLimitNs) {
-                    atomicOr(err, (unsigned long long)err_bit);
-                    return make_float4(NAN, 0.f, NAN, 0.f);
-                }
-            }
-        }
-        const float m = __uint_as_float((unsigned)r.x);
-        if (greedy) {
-            const unsigned lo = (unsigned)r.y;
-            return make_float4(m, 0.f, (lo >> 31) ? 1.f : 0.f, __int_as_float((int)(lo & 0x7fffffffu)));
-        }
-        const float mk = (m == -INFINITY) ? 0.f : ceilf(__fmul_rn(m, khi));
-        return make_float4(m, mk, __uint_as_float((unsigned)r.y), 0.f);
-    }
 };
 
 // Everything the per-sequence finish needs: logits for the gathers, the

@@ -72,18 +72,6 @@ __device__ __forceinline__ const unsigned char* row_ptr(const TailArgs& t, int b
                : static_cast<const unsigned char*>(t.dft) + ((size_t)b * t.gamma + (r - t.gamma - 1)) * V * ESZ;
 }
 
-// SeqRec written by another CTA: read at L2, after the fence that follows its flag.
-__device__ __forceinline__ SeqRec load_seqrec_cg(const SeqRec* p)
-{
-    union {
-        int4 v[2];
-        SeqRec r;
-    } u;
-    u.v[0] = __ldcg(reinterpret_cast<const int4*>(p));
-    u.v[1] = __ldcg(reinterpret_cast<const int4*>(p) + 1);
-    return u.r;
-}
-
 template <int ESZ>
 __device__ __forceinline__ uint4 neg_inf_vec()
 {
