@@ -18,7 +18,7 @@ def pytest_configure(config):
 
 def pytest_collection_modifyitems(config, items):
     # GPU tests are skipped, not failed, when no GPU is present and the user did not
-    # ask for them explicitly; with -m gpu on a GPU machine they run.
+    # ask for them explicitly; with -m gpu on a machine with a GPU they run.
     try:
         import torch
         has_gpu = torch.cuda.is_available()
