@@ -47,11 +47,12 @@ RAGGED = [
 
 # 16-byte-aligned rows of at least 4 KB: the streaming kernels.  Short rows (one
 # pass-1 span covers several), gamma = 32 (65 rows per sequence), a ragged last
-# tile, draws over more than one block of tile sums, and rows whose tile sums do
-# not fit in shared memory (more than 4096 tiles).
+# tile, draws over more than one block of tile sums, rows whose tile sums do not
+# fit in shared memory (more than 4096 tiles), and more sequences than resident
+# pass-2 clusters (each cluster finishes and draws several in turn).
 ALIGNED = [
     (5, 3, 2056, "bf16"), (2, 32, 1032, "f32"), (7, 4, 40008, "bf16"), (11, 6, 12344, "f32"),
-    (1, 2, 250000, "f32"), (3, 1, 600000, "f32"), (90, 2, 4096, "bf16"),
+    (1, 2, 250000, "f32"), (3, 1, 600000, "f32"), (90, 2, 4096, "bf16"), (400, 1, 2048, "bf16"),
 ]
 
 
