@@ -27,7 +27,10 @@
  *      "Amostragem Saguaro"]; after gamma acceptances it is the bonus token,
  *      drawn from the target's (gamma+1)-th distribution p_gamma.  The draw is
  *      an inverse CDF with u = u_resample[b]: the smallest token k whose running
- *      weight sum C_k exceeds u * (sum of all weights).
+ *      weight sum C_k exceeds u * (sum of all weights).  A residual whose total
+ *      mass is below 2^-18 counts as vanished (q_n equals p_n to within
+ *      rounding there, and the residual is then proportional to p_n): the token
+ *      is drawn from p_n and status bit SV_ROW_RESIDUAL_ZERO is set.
  * With T == 0 the step is greedy: x_j is accepted iff it is the first argmax of
  * target row j, and the extra token is the first argmax of target row n.  The
  * draft logits and the uniforms of such a sequence are not read.
@@ -72,12 +75,15 @@ typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
 #define SV_TEMPERATURE_MIN 1e-6f
 
 /* Per-sequence status bits written to out_row_status (data-dependent errors
- * never trap; they are reported here).  With bit 1, 2 or 4 the sequence emits
- * n_accepted = 0 and out_tokens all -1. */
+ * never trap; they are reported here).  With bit 1, 2, 4 or 16 the sequence
+ * emits n_accepted = 0 and out_tokens all -1. */
 #define SV_ROW_BAD_TOKEN 1        /* some draft token outside [0, V) */
 #define SV_ROW_BAD_LOGITS 2       /* a row that is read holds NaN or +inf, or is all -inf */
 #define SV_ROW_BAD_TEMPERATURE 4  /* T < 0, NaN, +inf, or 0 < T < SV_TEMPERATURE_MIN */
-#define SV_ROW_RESIDUAL_ZERO 8    /* residual mass was 0; the token was drawn from p_n */
+#define SV_ROW_RESIDUAL_ZERO 8    /* residual mass below 2^-18 (it counts as vanished);
+                                     the token was drawn from p_n instead */
+#define SV_ROW_BAD_UNIFORM 16     /* T > 0 and some u_accept[b][j] or u_resample[b]
+                                     outside [0, 1) or NaN */
 
 /*
  * Bytes of device workspace spec_verify() needs for this shape (0 on a bad
@@ -112,8 +118,8 @@ sv_status spec_verify_workspace_init(void* workspace, size_t workspace_bytes,
  *   draft_logits    [B][gamma][V]   of dt, contiguous, 16-byte aligned
  *   draft_tokens    [B][gamma] int32
  *   temperature     [B] float; 0 = greedy
- *   u_accept        [B][gamma] float, expected in (0, 1)
- *   u_resample      [B] float, expected in (0, 1)
+ *   u_accept        [B][gamma] float in [0, 1) (else status SV_ROW_BAD_UNIFORM)
+ *   u_resample      [B] float in [0, 1) (else status SV_ROW_BAD_UNIFORM)
  *   out_tokens      [B][gamma+1] int32: the n accepted drafts, the extra token,
  *                   then -1
  *   out_n_accepted  [B] int32 in [0, gamma]
@@ -154,9 +160,12 @@ const char* spec_verify_status_string(sv_status status);
  *  - Shapes whose workspace (spec_verify_workspace_size) exceeds
  *    SV_NOALLOC_SCRATCH_BYTES are rejected with SV_ERR_WORKSPACE_TOO_SMALL
  *    before anything is launched.
- *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current); make that first call before any stream
- *    capture begins.
+ *  - The first call in a CUDA context (a device's primary context, or a context
+ *    the caller made current) looks up the array's device address in that
+ *    context; make that first call before any stream capture begins.  The
+ *    address is cached per context under the context's unique ID, so after
+ *    cudaDeviceReset, or in another context, the next call looks it up again
+ *    rather than reusing an address that no longer belongs to it.
  *  - The call allocates nothing: it clears the completion counters with
  *    cudaMemsetAsync on `stream` and then launches the same kernels as
  *    spec_verify().

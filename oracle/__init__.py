@@ -22,7 +22,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "sv_oracle.c")
 _LIB = os.path.join(_HERE, "libsvoracle.so")
 
-ST_TOKEN, ST_ROW, ST_TEMP, ST_RESID0 = 1, 2, 4, 8
+ST_TOKEN, ST_ROW, ST_TEMP, ST_RESID0, ST_UNIFORM = 1, 2, 4, 8, 16
+RESIDUAL_MIN = 2.0 ** -18   # residual mass below this counts as vanished
 NEAR_ACCEPT, NEAR_CDF = 1, 2
 
 
@@ -67,7 +68,8 @@ class OracleResult:
     row_status: np.ndarray   # [B] int32 bitmask
     near_tie: np.ndarray     # [B] int32 bitmask (1 accept test, 2 inverse CDF)
     accept_gap: np.ndarray   # [B] float64: min |log u_j - delta_j| over tested j
-    cdf_gap: np.ndarray      # [B] float64: distance of u*S to the chosen bin's edges, / S
+    cdf_gap: np.ndarray      # [B] float64: distance of u*S to the chosen bin's edges (probability
+                             # units), or |S - RESIDUAL_MIN| after a rejection if smaller
 
 
 def max_threads() -> int:

@@ -26,8 +26,13 @@
  *     from the target's (gamma+1)-th distribution p_gamma.
  *     Inverse CDF: the token is the smallest k with C_k > u * S, where C_k is the
  *     running sum of the weights and S their total; if rounding leaves no such k,
- *     the last k with a positive weight.  If the residual is all zero, the draw
- *     falls back to p_n (row-status bit 8).
+ *     the last k with a positive weight.  If the residual mass S is below
+ *     2^-18 the residual counts as vanished and the draw falls back to p_n
+ *     (row-status bit 8).  S = 0 needs p_n <= q_n at every token, which with
+ *     both summing to one leaves only rounding-level differences; a mass this
+ *     small is also below what fp32 weights resolve, and in the cases that
+ *     reach it (q_n equal to p_n up to a shift of the normaliser) the residual
+ *     is proportional to p_n anyway.
  *  4. T == 0 is greedy verification: accept j iff x_j is the first argmax of
  *     target row j; the extra token is the first argmax of target row n.  The
  *     draft logits and the uniforms are not used.
@@ -40,15 +45,20 @@
  * Contract details that the pages leave open (library readings):
  *   - valid temperature: T == 0, or T finite and >= 1e-6; otherwise status 4;
  *   - status 1: some draft token outside [0, V);
+ *   - status 16 (T > 0 only): some uniform u_accept[j] or u_resample outside
+ *     [0, 1) or NaN (the uniforms stand for draws of U[0, 1));
  *   - status 2: a row that is read holds NaN or +inf, or is all -inf
  *     (T > 0: all 2*gamma+1 rows; T == 0: the gamma+1 target rows);
- *   - with status 1, 2 or 4 the sequence emits n = 0 and all tokens -1;
+ *   - with status 1, 2, 4 or 16 the sequence emits n = 0 and all tokens -1;
  *   - tokens past the extra one are -1;
  *   - log_norm is NaN for greedy sequences, invalid T and bad rows.
  *
  * Near-tie report (for comparing an implementation that rounds differently):
  *   bit 1: |log u_j - delta_j| < 1e-6 at some tested position j;
- *   bit 2: at the chosen token k, min(|C_{k-1} - uS|, |C_k - uS|) / S < 1e-6.
+ *   bit 2: at the chosen token k, min(|C_{k-1} - uS|, |C_k - uS|) < 1e-6, the
+ *          weights being probabilities (p_v, or max(0, p_v - q_v)), so the gap
+ *          is in units of probability mass; or, after a rejection, the residual
+ *          mass S lies within 1e-6 of the 2^-18 fallback threshold.
  *
  * Inputs: logits are float32, or bf16 given as uint16 bit patterns; every
  * value is widened exactly to double before any arithmetic.
@@ -63,8 +73,9 @@
 
 #define ORACLE_T_MIN 1e-6
 #define ORACLE_NEAR 1e-6
+#define ORACLE_RESIDUAL_MIN 0x1p-18 /* residual mass below this counts as vanished */
 
-enum { ST_TOKEN = 1, ST_ROW = 2, ST_TEMP = 4, ST_RESID0 = 8 };
+enum { ST_TOKEN = 1, ST_ROW = 2, ST_TEMP = 4, ST_RESID0 = 8, ST_UNIFORM = 16 };
 enum { NEAR_ACCEPT = 1, NEAR_CDF = 2 };
 
 static double widen(const void* base, int is_bf16, size_t i)
@@ -126,7 +137,7 @@ static int inverse_cdf(const double* w, int V, double u, int* near, double* gap)
         *gap = 0.0;
         return k;
     }
-    *gap = fmin(fabs(prev - target), fabs(C - target)) / S;
+    *gap = fmin(fabs(prev - target), fabs(C - target));
     if (*gap < ORACLE_NEAR) *near |= NEAR_CDF;
     return k;
 }
@@ -151,6 +162,11 @@ static void verify_one(const void* tgt, const void* dft, int is_bf16, const int3
     }
     for (int j = 0; j < gamma; ++j)
         if (tok[j] < 0 || tok[j] >= V) st |= ST_TOKEN;
+    if (T > 0.0) { /* a greedy sequence reads no uniform */
+        for (int j = 0; j < gamma; ++j)
+            if (!(u_acc[j] >= 0.0f && u_acc[j] < 1.0f)) st |= ST_UNIFORM;
+        if (!(u_res >= 0.0 && u_res < 1.0)) st |= ST_UNIFORM;
+    }
 
     const size_t trow0 = b * (size_t)(gamma + 1) * (size_t)V;
     const size_t drow0 = b * (size_t)gamma * (size_t)V;
@@ -209,12 +225,15 @@ static void verify_one(const void* tgt, const void* dft, int is_bf16, const int3
             wbuf[v] = fmax(0.0, p - q);
             S += wbuf[v];
         }
-        if (!(S > 0.0)) {
+        if (!(S >= ORACLE_RESIDUAL_MIN)) {
             st |= ST_RESID0;
             for (int v = 0; v < V; ++v)
                 wbuf[v] = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);
         }
         k = inverse_cdf(wbuf, V, u_res, &nr, cgap);
+        /* the fallback decision itself is a near tie when S is close to the threshold */
+        if (fabs(S - ORACLE_RESIDUAL_MIN) < *cgap) *cgap = fabs(S - ORACLE_RESIDUAL_MIN);
+        if (*cgap < ORACLE_NEAR) nr |= NEAR_CDF;
     } else {
         for (int v = 0; v < V; ++v)
             wbuf[v] = exp(widen(tgt, is_bf16, trow0 + (size_t)gamma * V + v) / T - lse_t[gamma]);
@@ -231,8 +250,9 @@ static void verify_one(const void* tgt, const void* dft, int is_bf16, const int3
  * target: [B][gamma+1][V], draft: [B][gamma][V]; is_bf16 selects uint16 bf16 bits.
  * Outputs: out_tokens [B][gamma+1], out_n [B], log_norm [B][2*gamma+1],
  * row_status [B], near_tie [B], accept_gap [B] (smallest |log u_j - delta_j| over
- * the tested positions), cdf_gap [B] (the inverse-CDF gap above; +inf when no draw
- * was made).  Returns 0, or -1 on a bad shape.
+ * the tested positions), cdf_gap [B] (the inverse-CDF gap above, or |S - 2^-18|
+ * after a rejection if that is smaller; +inf when no draw was made).  Returns 0,
+ * or -1 on a bad shape.
  */
 int sv_oracle_verify(const void* target, const void* draft, int is_bf16,
                      const int32_t* draft_tokens, const float* temperature,

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "lib", "libspecverify.so")
 
 SV_OK = 0
 SV_DTYPE_F32, SV_DTYPE_BF16 = 0, 1
-ROW_BAD_TOKEN, ROW_BAD_LOGITS, ROW_BAD_TEMPERATURE, ROW_RESIDUAL_ZERO = 1, 2, 4, 8
+ROW_BAD_TOKEN, ROW_BAD_LOGITS, ROW_BAD_TEMPERATURE, ROW_RESIDUAL_ZERO, ROW_BAD_UNIFORM = 1, 2, 4, 8, 16
 EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_init",
             "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc")
 # byte offset of the error word in a workspace (nonzero only if a bounded wait gave up)

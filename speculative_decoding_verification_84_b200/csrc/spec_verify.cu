@@ -12,6 +12,7 @@
 // every shape (both compute the same results; tests use it to cover both).
 #include "spec_verify.h"
 
+#include <cuda.h>  // CUcontext / CUresult types only: driver calls go through entry points
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -188,6 +189,7 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
     t.tokens = tokens;
     t.temperature = temperature;
     t.u_accept = u_acc;
+    t.u_resample = u_res;
     t.out_tokens = out_tokens;
     t.out_n = out_n;
     t.out_log_norm = out_ln;
@@ -357,28 +359,75 @@ extern "C" const char* spec_verify_status_string(sv_status s)
 // For callers that cannot allocate device memory (see spec_verify_noalloc in the
 // header): the workspace is this fixed array, one per GPU for the life of the
 // process.  Host code must not pass the symbol itself to a kernel (on the host it
-// names a stand-in, not device memory); its device address is looked up once per
-// device below.
+// names a stand-in, not device memory); its device address is looked up below.
+//
+// The address belongs to one CUDA context.  It is cached per context, keyed by
+// the context's unique ID (cuCtxGetId: never reused within a process), so a
+// context created later -- after cudaDeviceReset, or a caller's own context made
+// current -- gets a fresh lookup instead of a stale address.  The two driver
+// calls are reached through cudaGetDriverEntryPointByVersion, so the library
+// does not link against the driver library.
 
 static __device__ __align__(256) unsigned char sv_noalloc_scratch[SV_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+constexpr int kNoallocCache = 16;
 
-// Device address of sv_noalloc_scratch on the current device (first use per device
-// does the lookup).  Returns nullptr on a CUDA error.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+struct NoallocEntry {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+
+std::mutex g_noalloc_mu;
+NoallocEntry g_noalloc_cache[kNoallocCache] = {};
+int g_noalloc_next = 0;
+
+// Unique ID of the context current on this thread, or 0 if there is none or the
+// driver calls are unavailable.
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of sv_noalloc_scratch in the current context (the first use in a
+// context does the lookup, which also makes the runtime bind a context if none is
+// current).  Returns nullptr on a CUDA error.
 void* noalloc_scratch_address()
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, sv_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-        g_noalloc_ptr[dev] = p;
+    unsigned long long id = current_context_id();
+    if (id)
+        for (const NoallocEntry& e : g_noalloc_cache)
+            if (e.ctx_id == id) return e.ptr;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, sv_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    if (!id) id = current_context_id();  // the lookup may have bound the primary context
+    if (id) {                            // without an ID, look it up again on every call
+        g_noalloc_cache[g_noalloc_next] = NoallocEntry{id, p};
+        g_noalloc_next = (g_noalloc_next + 1) % kNoallocCache;
     }
-    return g_noalloc_ptr[dev];
+    return p;
 }
 }  // namespace
 

@@ -26,6 +26,11 @@ constexpr int kThreads = 256;            // threads that compute (generic CTA / 
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxRows = 2 * SV_MAX_GAMMA + 1;
 constexpr double kLn2 = 0.69314718055994530942;
+// A residual mass below this counts as vanished and the extra token is drawn
+// from p_n instead (row-status bit 8): at this size the residual is below what
+// fp32 weights resolve, and the cases that reach it (q_n equal to p_n up to a
+// shift of the normaliser) have a residual proportional to p_n.
+constexpr double kResidualMin = 0x1p-18;
 constexpr double kLog2e = 1.44269504088896340736;
 
 enum : int { kModeNone = 0, kModeResidual = 1, kModeBonus = 2 };
@@ -418,6 +423,7 @@ struct TailArgs {
     const int32_t* tokens;
     const float* temperature;
     const float* u_accept;
+    const float* u_resample;
     int32_t* out_tokens;
     int32_t* out_n;
     double* out_log_norm;
@@ -471,8 +477,20 @@ __device__ void sequence_tail(const TailArgs& a, int b, int tid, const READ& rea
     if (tval && !greedy) split_k(T, &khi_t, &klo_t);
 
     // the accept test's scalars, fetched first so their latency overlaps the combine
-    int x_j = -1;
+    int x_j = -1, bad_u = 0;
     double lt_j = 0.0, ld_j = 0.0, lu_j = 0.0;
+    if (warp == 0 && tval && !greedy) {
+        // the uniforms stand for draws of U[0, 1): anything else (NaN included)
+        // is an invalid input (a greedy sequence reads none)
+        if (lane < gamma) {
+            const float u = a.u_accept[(size_t)b * gamma + lane];
+            bad_u = !(u >= 0.f && u < 1.f);
+        }
+        if (lane == 0) {
+            const float u = a.u_resample[b];
+            bad_u |= !(u >= 0.f && u < 1.f);
+        }
+    }
     if (warp == 0 && lane < gamma && tval) {
         x_j = tok[lane];
         if (a.gath) {  // the streaming pass stored them: no load that waits for x_j
@@ -547,6 +565,7 @@ __device__ void sequence_tail(const TailArgs& a, int b, int tid, const READ& rea
             for (int r = lane; r < rows_used; r += 32) badrow |= s_bad[r];
             if (__any_sync(0xffffffffu, badtok)) st |= SV_ROW_BAD_TOKEN;
             if (__any_sync(0xffffffffu, badrow)) st |= SV_ROW_BAD_LOGITS;
+            if (__any_sync(0xffffffffu, bad_u)) st |= SV_ROW_BAD_UNIFORM;
         }
         int n = 0;
         if (st == 0) {

@@ -263,8 +263,8 @@ __device__ void sequence_draw(const GenericArgs& g, int b, const SeqRec& s, cons
         S += tot;
     }
     int flag = 0;
-    if (!(S > 0.0) && s.mode == kModeResidual) {
-        // the residual vanished (p == q up to rounding): draw from p_n instead
+    if (!(S >= kResidualMin) && s.mode == kModeResidual) {
+        // the residual vanished (below kResidualMin): draw from p_n instead
         flag = SV_ROW_RESIDUAL_ZERO;
         p_only = true;
         for (int c = 0; c < nc; ++c) {

@@ -359,8 +359,8 @@ __device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& 
     __syncthreads();
     bool p_only = bonus;
     int flag = 0;
-    if (!(s_S > 0.0) && !bonus) {
-        // the residual vanished (p == q up to rounding): draw from p_n instead
+    if (!(s_S >= kResidualMin) && !bonus) {
+        // the residual vanished (below kResidualMin): draw from p_n instead
         flag = SV_ROW_RESIDUAL_ZERO;
         p_only = true;
         tile_sums_strided<ESZ>(g, rec, true, tv, tv, ws, warp, kWarps);

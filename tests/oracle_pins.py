@@ -342,31 +342,108 @@ def check_bonus_distribution(verify, min_samples=10_000, alpha=0.01):
     assert D < 1.628 / math.sqrt(n)
 
 
+# ----------------------------------------------------------------- vanished residual
+
+RESIDUAL_MIN = 2.0 ** -18   # the contract's threshold: a smaller residual mass counts as vanished
+
+
+def vanished_residual_cases(V, seed=41):
+    """Rows whose residual at position 0 vanishes, with the uniforms to use.
+
+    Target and draft row 0 are equal except at one token x, and the draft token
+    at position 0 is x, whose log ratio is about -0.75 or -1, so u_accept = 0.75
+    rejects it (log 0.75 = -0.29).
+      (a) both logits at x sit ~100 below the rest: the normalisers of the two
+          rows agree to far below rounding, so p_v = q_v for v != x and p_x < q_x:
+          the residual mass S is 0;
+      (b) p_0 ~ 1.3e-6 and the draft raises logit 0 by 1 (x = 0): S = q_0 - p_0
+          ~ 2.2e-6, still more than 1e-6 below 2^-18.  u_resample is placed
+          1.6e-6 above p_0, inside q's first bin but past p's, so a draw from
+          q instead of p would return token 0.
+    Returns a list of (lt_row0, ld_row0, x, u_resample) in float32."""
+    rng = np.random.default_rng(seed)
+    base = (rng.standard_normal(V) * 1.5).astype(np.float32)
+    out = []
+    x = min(7, V - 1)
+    lt = base.copy(); lt[x] = np.float32(-100.0)
+    ld = base.copy(); ld[x] = np.float32(-99.25)
+    for u in (0.3, 0.6, 0.95):
+        out.append((lt, ld, x, np.float32(u)))
+    lse_rest = fsum_lse(base[1:], 1.0)
+    lt = base.copy(); lt[0] = np.float32(lse_rest + math.log(1.3e-6))
+    ld = lt.copy(); ld[0] = np.float32(float(lt[0]) + 1.0)
+    p0 = float(fsum_softmax(lt, 1.0)[0])
+    for u in (p0 + 1.6e-6, 0.4, 0.9):
+        out.append((lt, ld, 0, np.float32(u)))
+    return out
+
+
+def check_residual_vanished(verify):
+    """Residual mass below 2^-18 after a rejection: status 8, n = 0, and the token is
+    numpy.searchsorted(cumsum(p_0), u * sum(p_0), 'right') with p_0 from math.fsum
+    (Speculative Speculative Decoding, Desafios 2, "Amostragem Saguaro": the
+    residual; the fallback is the library's reading for a residual that vanished)."""
+    V, gamma, T = 40, 2, 1.0
+    rng = np.random.default_rng(43)
+    cases = vanished_residual_cases(V)
+    B = len(cases)
+    tgt = (rng.standard_normal((B, gamma + 1, V)) * 1.5).astype(np.float32)
+    dft = (rng.standard_normal((B, gamma, V)) * 1.5).astype(np.float32)
+    toks = rng.integers(0, V, size=(B, gamma))
+    ur = np.empty(B, np.float32)
+    for i, (lt, ld, x, u) in enumerate(cases):
+        tgt[i, 0], dft[i, 0], toks[i, 0], ur[i] = lt, ld, x, u
+    ua = np.full((B, gamma), 0.75, np.float32)
+    r = verify(*_seq_batch(tgt, dft, toks, np.full(B, T), ua, ur))
+    for i, (lt, ld, x, u) in enumerate(cases):
+        p = fsum_softmax(lt.astype(np.float64), T)
+        q = fsum_softmax(ld.astype(np.float64), T)
+        S = math.fsum(np.maximum(0.0, p - q))
+        assert S < RESIDUAL_MIN - 1e-6, (i, S)          # the construction itself
+        C = np.cumsum(p)
+        target = float(u) * C[-1]
+        k = int(np.searchsorted(C, target, side="right"))
+        lo = C[k - 1] if k > 0 else 0.0
+        assert min(target - lo, C[k] - target) > 1e-6, i  # a clean draw, not a near tie
+        assert r.row_status[i] == 8, (i, r.row_status[i])
+        assert r.n_accepted[i] == 0, i
+        assert list(r.out_tokens[i]) == [k] + [-1] * gamma, (i, k, r.out_tokens[i])
+        assert r.cdf_gap[i] >= 1e-6, (i, r.cdf_gap[i])
+
+
 # ----------------------------------------------------------------- contract edges
 
 def check_status_edges(verify):
-    """Invalid temperature -> 4; token out of range -> 1; NaN/+inf/all -inf row -> 2."""
+    """Invalid temperature -> 4; token out of range -> 1; NaN/+inf/all -inf row -> 2;
+    a uniform outside [0, 1) or NaN -> 16 (T > 0 only: a greedy sequence reads none)."""
     V, gamma = 16, 2
     rng = np.random.default_rng(2)
     base_t = rng.standard_normal((gamma + 1, V)).astype(np.float32)
     base_d = rng.standard_normal((gamma, V)).astype(np.float32)
+    ok_u = ([0.5, 0.5], 0.5)
     cases = []
     for T in (-1.0, np.nan, np.inf, 1e-7):
-        cases.append((base_t, base_d, [1, 2], T, 4))
-    cases.append((base_t, base_d, [1, V], 1.0, 1))
-    cases.append((base_t, base_d, [-1, 0], 0.0, 1))
+        cases.append((base_t, base_d, [1, 2], T, 4, ok_u))
+    cases.append((base_t, base_d, [1, V], 1.0, 1, ok_u))
+    cases.append((base_t, base_d, [-1, 0], 0.0, 1, ok_u))
     bad = base_t.copy(); bad[1, 3] = np.nan
-    cases.append((bad, base_d, [1, 2], 1.0, 2))
-    cases.append((bad, base_d, [1, 2], 0.0, 2))
+    cases.append((bad, base_d, [1, 2], 1.0, 2, ok_u))
+    cases.append((bad, base_d, [1, 2], 0.0, 2, ok_u))
     bad = base_d.copy(); bad[0, :] = -np.inf
-    cases.append((base_t, bad, [1, 2], 1.0, 2))
-    cases.append((base_t, bad, [1, 2], 0.0, 0))   # greedy never reads draft rows
+    cases.append((base_t, bad, [1, 2], 1.0, 2, ok_u))
+    cases.append((base_t, bad, [1, 2], 0.0, 0, ok_u))   # greedy never reads draft rows
     bad = base_t.copy(); bad[2, 5] = np.inf
-    cases.append((bad, base_d, [1, 2], 1.0, 2))
-    for tg, dg, tk, T, st in cases:
-        r = verify(*_seq_batch(tg[None], dg[None], [tk], [T], [[0.5, 0.5]], [0.5]))
-        assert r.row_status[0] == st, (T, tk, st, r.row_status[0])
-        if st & 7:
+    cases.append((bad, base_d, [1, 2], 1.0, 2, ok_u))
+    for ua, ur in (([1.0, 0.5], 0.5), ([np.nan, 0.5], 0.5), ([0.5, -0.25], 0.5), ([0.5, 0.5], 1.0),
+                   ([0.5, 0.5], np.nan), ([0.5, 0.5], np.inf)):
+        cases.append((base_t, base_d, [1, 2], 1.0, 16, (ua, ur)))
+    cases.append((base_t, base_d, [1, V], 1.0, 17, ([2.0, 0.5], 0.5)))
+    cases.append((base_t, base_d, [1, 2], 1.0, 0, ([0.0, 0.0], 0.0)))   # 0 is in [0, 1)
+    cases.append((base_t, base_d, [1, 2], 0.0, 0, ([1.0, np.nan], 7.0)))  # greedy reads no uniform
+    for tg, dg, tk, T, st, (ua, ur) in cases:
+        r = verify(*_seq_batch(tg[None], dg[None], [tk], [T], [ua], [ur]))
+        assert r.row_status[0] == st, (T, tk, st, r.row_status[0], ua, ur)
+        if st & 23:
             assert r.n_accepted[0] == 0 and (r.out_tokens[0] == -1).all()
         if st == 4 or T == 0.0:
             assert np.isnan(r.log_norm[0]).all()
@@ -403,5 +480,5 @@ def check_output_invariants(verify):
 ALL_ORACLE_CHECKS = [
     check_lse_constant_rows, check_lse_shift_invariance, check_lse_fsum, check_masked_vocab,
     check_greedy_argmax, check_accept_boundary, check_inverse_cdf_searchsorted,
-    check_oracle_partition, check_status_edges, check_output_invariants,
+    check_residual_vanished, check_oracle_partition, check_status_edges, check_output_invariants,
 ]

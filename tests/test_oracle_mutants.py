@@ -33,6 +33,16 @@ MUTANTS = {
     "greedy_last_argmax": ("if (l > best) { best = l; arg = v; }", "if (l >= best) { best = l; arg = v; }"),
     "scan_past_first_rejection": ("if (!(lu < delta)) { n = j; break; }", "if (!(lu < delta)) { n = j; }"),
     "cdf_not_scaled_by_total": ("double target = u * S;", "double target = u;"),
+    "residual_fallback_removed": ("if (!(S >= ORACLE_RESIDUAL_MIN)) {", "if (0) {"),
+    "residual_fallback_draws_from_q": (
+        "                wbuf[v] = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);",
+        "                wbuf[v] = exp(widen(dft, is_bf16, drow0 + (size_t)n * V + v) / T - lse_d[n]);"),
+    "residual_fallback_next_row": (
+        "                wbuf[v] = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);",
+        "                wbuf[v] = exp(widen(tgt, is_bf16, trow0 + (size_t)(n + 1) * V + v) / T - lse_t[n + 1]);"),
+    "residual_fallback_unflagged": ("st |= ST_RESID0;", ";"),
+    "residual_threshold_zero": ("!(S >= ORACLE_RESIDUAL_MIN)", "!(S > 0.0)"),
+    "accept_uniform_unchecked": ("if (!(u_acc[j] >= 0.0f && u_acc[j] < 1.0f)) st |= ST_UNIFORM;", ";"),
     "draft_normaliser_for_target": (
         "double lp = widen(tgt, is_bf16, trow0 + (size_t)j * V + (size_t)tok[j]) / T - lse_t[j];",
         "double lp = widen(tgt, is_bf16, trow0 + (size_t)j * V + (size_t)tok[j]) / T - lse_d[j];"),

@@ -28,14 +28,14 @@ def test_config_full(name):
     parity.assert_parity(st)
 
 
-def test_config_c4_full_size_sampled():
-    """c4 at full size (B=256, gamma=8, V=151936) on the GPU; the oracle checks a
-    sample of sequences from every temperature class (greedy, 0.6, 1.0)."""
+def test_config_c4_full():
+    """c4 at full size (B=256, gamma=8, V=151936, greedy / 0.6 / 1.0 by sequence):
+    every sequence compared with the oracle."""
     w = W.make_workload("c4")
     g = parity.run_gpu(w)
-    idx = list(range(0, 256, 7)) + [253, 254, 255]
-    st = parity.compare(g, oracle.verify_workload(w.subset(idx)), idx=np.array(idx))
+    st = parity.compare(g, oracle.verify_workload(w))
     _report("c4", st)
+    assert st["B"] == 256
     parity.assert_parity(st)
 
 
@@ -79,10 +79,13 @@ def test_aligned_shapes(B, gamma, V, dt):
 
 @pytest.mark.parametrize("V", [300, 4096])
 def test_edge_cases(V):
-    """NaN / +inf / all -inf rows, out-of-range tokens, invalid temperatures, masked vocab
+    """NaN / +inf / all -inf rows, out-of-range tokens, invalid temperatures, masked vocab,
+    uniforms outside [0, 1), and residuals that vanish after a rejection
     (V = 300: the general kernels; V = 4096 f32, 16 KB rows: the streaming kernels)."""
+    import oracle_pins
     rng = np.random.default_rng(9)
-    B, gamma = 14, 3
+    vanished = oracle_pins.vanished_residual_cases(V)
+    B, gamma = 20 + len(vanished), 3
     tgt = (rng.standard_normal((B, gamma + 1, V)) * 2).astype(np.float32)
     dft = (tgt[:, :gamma] + rng.standard_normal((B, gamma, V))).astype(np.float32)
     toks = rng.integers(0, V, (B, gamma)).astype(np.int32)
@@ -101,10 +104,22 @@ def test_edge_cases(V):
     tgt[11, 0, :] = 1.0                        # all-tie greedy row: index 0 wins
     toks[11, 0] = 0
     tgt[12, 0, :] = -np.inf                    # all -inf row
-    w = W.Workload(f"edges-{V}", "f32", tgt, dft, toks, T, W.draw_uniforms(rng, (B, gamma)),
-                   W.draw_uniforms(rng, (B,)))
+    ua, ur = W.draw_uniforms(rng, (B, gamma)), W.draw_uniforms(rng, (B,))
+    ua[14, 0] = 1.0                            # uniforms outside [0, 1): status 16
+    ua[15, 1] = np.nan
+    ur[16] = 1.0
+    ur[17] = -0.5
+    ua[18, :], ur[18] = 0.0, 0.0               # 0 is a valid uniform
+    T[19], ua[19, 0], ur[19] = 0.0, 1.0, 2.0   # greedy reads no uniform
+    for i, (lt, ld, x, u) in enumerate(vanished):
+        b = 20 + i                             # the residual vanishes at position 0: status 8
+        tgt[b, 0], dft[b, 0], toks[b, 0], ua[b, 0], ur[b] = lt, ld, x, 0.75, u
+    w = W.Workload(f"edges-{V}", "f32", tgt, dft, toks, T, ua, ur)
     ref = oracle.verify_workload(w)
     assert ref.row_status[:9].tolist() == [2, 2, 2, 1, 1, 4, 4, 4, 4]
+    assert ref.row_status[14:20].tolist() == [16, 16, 16, 16, 0, 0]
+    assert (ref.row_status[20:] == 8).all() and (ref.n_accepted[20:] == 0).all()
+    assert (ref.cdf_gap[20:] >= parity.BAND).all()   # compared exactly, status bit 8 included
     st = parity.compare(parity.run_gpu(w), ref)
     _report(f"edges-{V}", st)
     parity.assert_parity(st)

@@ -43,15 +43,25 @@ def _call_noalloc(d, B, gamma, V, dt_code):
     return out_t, out_n, ln, st
 
 
-@pytest.mark.parametrize("first,second", [("c2", "mixed"), ("c3", "c2")])
+CASES = {
+    "c2": lambda: W.make_workload("c2"),
+    "c3": lambda: W.make_workload("c3"),
+    "mixed": lambda: W.make_random(19, 6, 5003, "f32", seed=1234, T=([0.0, 0.8, 1.0, 1.3] * 5)[:19]),
+    # the general kernels with a larger batch: its completion counters lie where the
+    # previous call ("mixed") left its per-sequence records, so they start nonzero
+    # unless the call clears them
+    "mixed_wide_batch": lambda: W.make_random(300, 2, 1001, "bf16", seed=4321, T=([0.0, 0.7, 1.0] * 100)),
+    # the streaming kernels with rows of more than 4096 tiles: tile sums in the
+    # scratch rather than in shared memory
+    "long_rows": lambda: W.make_random(2, 1, 600000, "f32", seed=99, T=[1.0, 0.8]),
+}
+
+
+@pytest.mark.parametrize("first,second", [("c2", "mixed"), ("c3", "c2"), ("mixed", "mixed_wide_batch"),
+                                          ("long_rows", "mixed_wide_batch")])
 def test_noalloc_matches_spec_verify_two_calls(first, second):
-    cases = {
-        "c2": lambda: W.make_workload("c2"),
-        "c3": lambda: W.make_workload("c3"),
-        "mixed": lambda: W.make_random(19, 6, 5003, "f32", seed=1234, T=([0.0, 0.8, 1.0, 1.3] * 5)[:19]),
-    }
     for name in (first, second):                     # two calls in a row share the scratch
-        w = cases[name]()
+        w = CASES[name]()
         tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         assert binding.workspace_size(w.B, w.gamma, w.V, tdt) <= NOALLOC_SCRATCH_BYTES
         d = binding.to_device(w)
