@@ -201,8 +201,8 @@ def run_ours(args):
     dt_code = binding._dt_code(tdt)
     kernels_per_call = binding.kernels_per_call(B, gamma, V, tdt)
     rowbytes = V * esz
-    kernel_name = ("sv_pass1 + sv_pass2 (one call; pass 1 streams every logit once)"
-                   if rowbytes % 16 == 0 and rowbytes >= 4096 else "sv_rowpass + sv_resample (one call)")
+    kernel_name = ("sv_stream + sv_draw (one call; sv_stream reads every logit once)"
+                   if rowbytes % 16 == 0 and rowbytes >= 4096 else "sv_reset + sv_rowpass + sv_resample (one call)")
 
     def call(d):
         st = lib.spec_verify(d["target"].data_ptr(), d["draft"].data_ptr(), dt_code, d["draft_tokens"].data_ptr(),

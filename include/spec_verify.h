@@ -88,22 +88,25 @@ typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
 /*
  * Bytes of device workspace spec_verify() needs for this shape (0 on a bad
  * shape).  The workspace is caller-owned device memory, 256-byte aligned.
+ * Infrastructure of this library: no passage of the pages stands behind it.
  *
- * Zero the whole workspace once after allocating it (for example with
- * spec_verify_workspace_init).  It then serves any number of calls with the same
- * (B, gamma, V, dt): every call that runs to completion leaves it ready for the
- * next.  Zero it again before reusing it for another shape.  Calls that share a
- * workspace must be ordered (same stream, or events).  The 8 bytes at offset 16
- * are reserved as an error word for kernels that wait on one another; the
- * kernels of this version never do, so it stays zero.
+ * The workspace needs no initialisation and keeps nothing between calls: a call
+ * reads no byte of it that the same call has not written first (the general
+ * kernels' per-sequence tickets are zeroed by the call's first launch), so any
+ * contents -- another shape's leftovers, garbage -- are fine.  Calls that share
+ * a workspace must be ordered (same stream, or events).  No kernel of either
+ * family waits on another, so there is no timeout or error word.
  */
 size_t spec_verify_workspace_size(int B, int gamma, int V, sv_dtype dt);
 
-/* Number of kernel launches one spec_verify() call of this shape enqueues (2
- * for either kernel family), or 0 on a bad shape. */
+/* Number of kernel launches one spec_verify() call of this shape enqueues (3:
+ * the counter reset, then one streaming kernel or two general kernels), or 0 on
+ * a bad shape.  Infrastructure: no passage of the pages stands behind it. */
 int spec_verify_kernels_per_call(int B, int gamma, int V, sv_dtype dt);
 
-/* cudaMemsetAsync(workspace, 0, workspace_bytes, stream). */
+/* cudaMemsetAsync(workspace, 0, workspace_bytes, stream).  Not required before
+ * spec_verify (see spec_verify_workspace_size); kept for callers that want a
+ * known state.  Infrastructure: no passage of the pages stands behind it. */
 sv_status spec_verify_workspace_init(void* workspace, size_t workspace_bytes,
                                      struct CUstream_st* stream);
 
@@ -141,7 +144,8 @@ sv_status spec_verify(const void* target_logits, const void* draft_logits, sv_dt
                       double* out_log_norm, int32_t* out_row_status,
                       struct CUstream_st* stream);
 
-/* Static description of a status code; never NULL. */
+/* Static description of a status code; never NULL.  Infrastructure: no passage
+ * of the pages stands behind it. */
 const char* spec_verify_status_string(sv_status status);
 
 /*
@@ -166,9 +170,8 @@ const char* spec_verify_status_string(sv_status status);
  *    address is cached per context under the context's unique ID, so after
  *    cudaDeviceReset, or in another context, the next call looks it up again
  *    rather than reusing an address that no longer belongs to it.
- *  - The call allocates nothing: it clears the completion counters with
- *    cudaMemsetAsync on `stream` and then launches the same kernels as
- *    spec_verify().
+ *  - The call allocates nothing: it launches the same kernels as spec_verify()
+ *    on `stream`, the first of which zeroes the counters in the array.
  *  - Every call shares the one array and leaves its contents behind, so calls
  *    that overlap on the GPU (different streams without ordering, or several
  *    host threads) race and give wrong results.  Order them.

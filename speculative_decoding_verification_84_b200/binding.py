@@ -21,8 +21,6 @@ SV_DTYPE_F32, SV_DTYPE_BF16 = 0, 1
 ROW_BAD_TOKEN, ROW_BAD_LOGITS, ROW_BAD_TEMPERATURE, ROW_RESIDUAL_ZERO, ROW_BAD_UNIFORM = 1, 2, 4, 8, 16
 EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_init",
             "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc")
-# byte offset of the error word in a workspace (nonzero only if a bounded wait gave up)
-WORKSPACE_ERROR_OFFSET = 16
 
 _lib = None
 
@@ -79,17 +77,13 @@ def kernels_per_call(B: int, gamma: int, V: int, dtype: torch.dtype) -> int:
     return int(load_library().spec_verify_kernels_per_call(B, gamma, V, _dt_code(dtype)))
 
 
-def workspace_error(ws: torch.Tensor) -> int:
-    """The workspace's error word (0 unless a bounded device wait gave up)."""
-    return int(ws[WORKSPACE_ERROR_OFFSET:WORKSPACE_ERROR_OFFSET + 8].cpu().view(torch.int64).item())
-
-
 _ws_cache: Dict[Tuple, torch.Tensor] = {}
 
 
 def workspace_for(B: int, gamma: int, V: int, dtype: torch.dtype, device) -> torch.Tensor:
-    """A zero-initialised workspace cached per (device, shape).  Calls that share it
-    must be ordered on one stream; pass ``workspace=`` to run shapes concurrently."""
+    """A workspace cached per (device, shape); it needs no initialisation.  Calls
+    that share it must be ordered on one stream; pass ``workspace=`` to run shapes
+    concurrently."""
     device = torch.device(device)
     key = (device.index, B, gamma, V, dtype)
     ws = _ws_cache.get(key)

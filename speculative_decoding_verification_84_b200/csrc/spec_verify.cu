@@ -2,12 +2,14 @@
 // The operation is specified in include/spec_verify.h.  This file plans a call
 // (which kernel family, how the vocabulary is split, where everything lives in
 // the workspace) and launches it:
-//   * sv_pass1 + sv_pass2 (sv_pass.cuh): two persistent kernels; pass 1 gives
-//     every warp one contiguous span of the row stream, pass 2 finishes the
-//     sequences and then sums and draws from the residual rows.  Used when every
+//   * sv_stream + sv_draw (sv_pass.cuh): a persistent streaming kernel that
+//     reads every logit once, then a programmatic dependent that finishes each
+//     sequence, sums its draw rows (mostly from L2) and draws.  Used when every
 //     row is 16-byte aligned (V * element size a multiple of 16) and at least
-//     4 KB long.
-//   * sv_rowpass + sv_resample (sv_generic.cuh): any shape.
+//     4 KB long.  Every slot these kernels read, the same call wrote.
+//   * sv_reset + sv_rowpass + sv_resample (sv_generic.cuh): any shape; sv_reset
+//     zeroes the per-sequence tickets first, so a workspace carries nothing from
+//     one call to the next.
 // SPEC_VERIFY_FORCE_GENERIC=1 in the environment selects the second family for
 // every shape (both compute the same results; tests use it to cover both).
 #include "spec_verify.h"
@@ -34,15 +36,22 @@ constexpr int kPass1MinChunk = 1024;      // generic: elements
 constexpr int kPass2Chunk = 8192;         // generic: elements per residual CTA
 constexpr int kPass2MinChunk = 512;
 constexpr int kMaxDevices = 64;
+// streaming path: the last rows streamed that are meant to stay in L2 for the
+// draw (the rest load with an evict-first hint); about 2/3 of the 126 MB L2
+constexpr long long kL2KeepBytes = 80LL << 20;
 
 struct Plan {
     int B, gamma, V, R, esz;
     bool stream;
     int nc1, C1, nc2, C2;           // generic
     int nslot, NT2;                 // stream
+    long long evict_rows;           // stream: rows loaded evict-first
     long long nq;                   // stream: 16-byte vectors per row
     long long rowbytes;
-    size_t off_cnt, off_t1, off_t2, off_seq, off_gath, off_part, off_rsum, total;
+    // workspace: [0, off_seq) holds the general path's tickets (zeroed by that
+    // path at the start of every call); the rest is written by a call before the
+    // same call reads it
+    size_t off_c32a, off_c32b, off_seq, off_gath, off_part, off_rsum, total;
 };
 
 __host__ inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -88,21 +97,20 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     p->C2 = (int)((cdiv(V, nc2) + 7) / 8 * 8);
     p->nc2 = (int)cdiv(V, p->C2);
 
-    // streaming split: pass-1 spans of at least kSpanMin vectors (so a row meets
-    // at most nslot of them), 512-byte tiles for the draw
+    // streaming split: every warp span meets a row at most kStreamSlots times;
+    // 512-byte tiles for the draw; the last kL2KeepBytes of the stream stay in L2
     p->nq = p->rowbytes / 16;
-    p->nslot = (int)cdiv(p->nq, kSpanMin) + 1;
+    p->nslot = kStreamSlots;
     p->NT2 = (int)cdiv(p->nq, kTileVecs);
+    p->evict_rows = std::max<long long>(0, rows - kL2KeepBytes / p->rowbytes);
 
     // stream: one Partial per (row, span) slot; one float per tile (two per 8-byte slot)
     const long long nparts = rows * (p->stream ? (long long)p->nslot : p->nc1);
     const long long nrsum = p->stream ? cdiv((long long)B * p->NT2, 2) : (long long)B * p->nc2;
     size_t off = 0;
-    p->off_cnt = off;
-    off += 4 * sizeof(unsigned long long);
-    p->off_t1 = off;
+    p->off_c32a = off;  // general path: row-pass ticket per sequence
     off += sizeof(unsigned) * (size_t)B;
-    p->off_t2 = off;
+    p->off_c32b = off;  // general path: resample ticket per sequence
     off += sizeof(unsigned) * (size_t)B;
     off = align256(off);
     p->off_seq = off;
@@ -150,7 +158,7 @@ int ctas_per_sm(K kernel, int slot)
     return cache[slot][dev];
 }
 
-// Clusters of cs CTAs of sv_pass2 that can be resident at once on the current
+// Clusters of cs CTAs of sv_draw that can be resident at once on the current
 // device (cached per cluster size and device; 0 on a CUDA error).
 template <int ESZ>
 int max_clusters(int cs)
@@ -172,7 +180,7 @@ int max_clusters(int cs)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, sv_pass2<ESZ>, &cfg) != cudaSuccess || n < 1) n = -1;
+        if (cudaOccupancyMaxActiveClusters(&n, sv_draw<ESZ>, &cfg) != cudaSuccess || n < 1) n = -1;
         cache[cs][dev] = n;
     }
     return cache[cs][dev];
@@ -194,7 +202,7 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
     t.out_n = out_n;
     t.out_log_norm = out_ln;
     t.out_status = out_st;
-    t.ticket = reinterpret_cast<unsigned*>(ws + p.off_t1);
+    t.ticket = reinterpret_cast<unsigned*>(ws + p.off_c32a);
     t.seq = reinterpret_cast<SeqRec*>(ws + p.off_seq);
     t.part = reinterpret_cast<const Partial*>(ws + p.off_part);
     t.gath = nullptr;
@@ -208,27 +216,29 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
         g.part = reinterpret_cast<Partial*>(ws + p.off_part);
         g.gath = reinterpret_cast<float*>(ws + p.off_gath);
         g.t.gath = g.gath;
+        g.t.nc = kStreamSlots;
+        g.t.part = g.part;
         g.tsum = reinterpret_cast<float*>(ws + p.off_rsum);
         g.u_resample = u_res;
         g.nq = p.nq;
         g.NT2 = p.NT2;
         g.B = p.B;
-        // pass 1: as many CTAs as are resident at once, the row stream split into
-        // one span per warp
-        const int c1 = ctas_per_sm(sv_pass1<ESZ>, ESZ == 2 ? 0 : 1);
+        g.evict_rows = p.evict_rows;
+        // sv_stream: as many CTAs as are resident at once, the row stream split into
+        // one span per warp, each at least nq/31 vectors (a row meets at most
+        // kStreamSlots spans)
+        const int c1 = ctas_per_sm(sv_stream<ESZ>, ESZ == 2 ? 0 : 1);
         if (c1 < 1) return cudaErrorInvalidConfiguration;
         const long long sms = device_sm_count();
         const long long NQ = (long long)p.B * p.R * p.nq;
-        long long grid1 = sms * c1;
-        g.S = std::max<long long>(kSpanMin, cdiv(NQ, grid1 * kWarps));
-        grid1 = std::min<long long>(grid1, cdiv(cdiv(NQ, g.S), kWarps));
-        // a row meets at most this many spans: the partial slots per row
-        g.t.nc = (int)(cdiv(p.nq, g.S) + 1);
-        sv_pass1<ESZ><<<(unsigned)grid1, kPassThreads, 0, st>>>(g);
+        const long long nw = sms * c1 * kWarps;
+        g.S = std::max(std::max<long long>(kStreamSpanMin, cdiv(p.nq, kStreamSlots - 1)), cdiv(NQ, nw));
+        const long long grid1 = std::min<long long>(sms * c1, cdiv(cdiv(NQ, g.S), kWarps));
+        sv_stream<ESZ><<<(unsigned)grid1, kPassThreads, 0, st>>>(g);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
 
-        // pass 2: clusters of cs CTAs, one per sequence at a time; the largest
+        // sv_draw: clusters of cs CTAs, one sequence at a time each; the largest
         // cs (<= kMaxCluster) for which one wave of resident clusters covers the
         // batch, else 1
         int cs = 1, nclusters = 0;
@@ -243,8 +253,8 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
         }
         if (nclusters < 1) return cudaErrorInvalidConfiguration;
         const long long grid2 = (long long)cs * std::min<long long>(nclusters, p.B);
-        // a programmatic dependent launch: pass 2 may start while pass 1's last
-        // CTAs run, and waits on the device for pass 1's completion
+        // a programmatic dependent launch: sv_draw's CTAs start as sv_stream's
+        // leave, and wait on the device for sv_stream's completion
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid2);
         cfg.blockDim = dim3(kPassThreads);
@@ -259,9 +269,17 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
         attr[1].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
-        return cudaLaunchKernelEx(&cfg, sv_pass2<ESZ>, g);
+        return cudaLaunchKernelEx(&cfg, sv_draw<ESZ>, g);
     }
 
+    // general path: zero the tickets, then the two kernels
+    {
+        const long long n16 = (long long)(p.off_seq / 16);
+        const int gr = (int)std::min<long long>(cdiv(n16, 256), device_sm_count());
+        sv_reset<<<gr, 256, 0, st>>>(reinterpret_cast<uint4*>(ws), n16);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     GenericArgs g;
     g.t = t;
     g.t.nc = p.nc1;
@@ -269,7 +287,7 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
     g.nc1 = p.nc1;
     g.C1 = p.C1;
     g.u_resample = u_res;
-    g.ticket2 = reinterpret_cast<unsigned*>(ws + p.off_t2);
+    g.ticket2 = reinterpret_cast<unsigned*>(ws + p.off_c32b);
     g.rsum = reinterpret_cast<double*>(ws + p.off_rsum);
     g.nc2 = p.nc2;
     g.C2 = p.C2;
@@ -299,7 +317,7 @@ extern "C" int spec_verify_kernels_per_call(int B, int gamma, int V, sv_dtype dt
 {
     Plan p;
     if (!make_plan(B, gamma, V, dt, &p)) return 0;
-    return 2;
+    return p.stream ? 2 : 3;  // sv_stream + sv_draw, or sv_reset + sv_rowpass + sv_resample
 }
 
 extern "C" sv_status spec_verify_workspace_init(void* workspace, size_t workspace_bytes,
@@ -451,9 +469,8 @@ extern "C" sv_status spec_verify_noalloc(const void* target_logits, const void* 
     unsigned char* ws = static_cast<unsigned char*>(noalloc_scratch_address());
     if (!ws) return SV_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
-    // what must start at zero: the error word and the general path's tickets
-    // (every call leaves them zero, but the array is shared by every shape)
-    if (cudaMemsetAsync(ws, 0, p.off_seq, st) != cudaSuccess) return SV_ERR_CUDA;
+    // a call reads nothing it has not written first (the general kernels' tickets
+    // are zeroed by its first launch), as for any workspace
     const cudaError_t e =
         dt == SV_DTYPE_BF16
             ? launch<2>(p, target_logits, draft_logits, draft_tokens, temperature, u_accept, u_resample, out_tokens,

@@ -278,6 +278,64 @@ __device__ __forceinline__ void lse_fold(Lse& a, const float* acc)
     a.s += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
+// ---- online log-sum-exp with a lagging offset
+//
+// The streaming pass keeps, per warp, one offset mk (an integer, carried from
+// segment to segment) and per-lane accumulators of 2^(l*k - mk) on packed fp32
+// pairs.  Unlike lse_group2 it takes no maximum in the loop: every term is formed
+// against the offset already held.  The segment's sum is checked once at its
+// end: outside [2^-40, 2^100) (a term far above the offset or an overflow, a
+// carried offset far above this row's values, NaN, an all -inf segment) the
+// segment is summed again exactly (maximum first) -- rare, and the data is then
+// mostly in L2.  Inside that range no term overflowed and terms down to 2^-126
+// against the offset (at most 2^-86 of the sum) were kept, so the relative
+// precision is that of the exact form.
+
+// Exponentials of NV vectors against offset mk, added into 4 packed pairs acc.
+// bf16: word w of a vector holds elements 2w, 2w+1 -> pair w.  fp32: elements
+// (0,1) and (2,3) of vector u -> pairs 2(u&1), 2(u&1)+1.
+template <int ESZ, int NV>
+__device__ __forceinline__ void lazy_exps_add(unsigned long long* acc, const uint4* v, float khi, float klo, float mk)
+{
+    const unsigned long long KH = pack2(khi, khi), KL = pack2(klo, klo), NM = pack2(-mk, -mk);
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const unsigned wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        if (ESZ == 2) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const unsigned long long x2 = pack2(bf16_lo(wd[w]), bf16_hi(wd[w]));
+                const unsigned long long y2 = fma2(x2, KL, fma2(x2, KH, NM));
+                float y0, y1;
+                unpack2(y2, y0, y1);
+                acc[w] = add2(acc[w], pack2(ex2(y0), ex2(y1)));
+            }
+        } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const unsigned long long x2 = pack2(__uint_as_float(wd[2 * h]), __uint_as_float(wd[2 * h + 1]));
+                const unsigned long long y2 = fma2(x2, KL, fma2(x2, KH, NM));
+                float y0, y1;
+                unpack2(y2, y0, y1);
+                const int w = (u & 1) * 2 + h;
+                acc[w] = add2(acc[w], pack2(ex2(y0), ex2(y1)));
+            }
+        }
+    }
+}
+
+// Sum of a warp's accumulators (all lanes against the same offset), in every lane.
+__device__ __forceinline__ float lazy_warp_sum(const unsigned long long* acc)
+{
+    float a[8];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) unpack2(acc[w], a[2 * w], a[2 * w + 1]);
+    float s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+
 // 2^d in double for an integer-valued d <= 0 (exact; 0 below the normal range)
 __device__ __forceinline__ double pow2d(float d)
 {
@@ -622,7 +680,6 @@ __device__ void sequence_tail(const TailArgs& a, int b, int tid, const READ& rea
         }
         a.seq[b] = rec;
         sm.rec = rec;
-        a.ticket[b] = 0u;  // every contribution has arrived: ready for the next call
     }
 }
 

@@ -31,6 +31,15 @@ struct GenericArgs {
     int nc2, C2;
 };
 
+// Zero the call's tickets (n 16-byte words).  The general path
+// counts arrivals per sequence; starting every call from zero means a workspace
+// carries nothing from one call to the next.
+__global__ void __launch_bounds__(256) sv_reset(uint4* p, long long n)
+{
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 template <int ESZ, bool GREEDY>
 __device__ __forceinline__ void scan_chunk(const unsigned char* rowp, int v0, int v1, float khi,
                                            float klo, Lse& L, Amax& A)
@@ -349,7 +358,6 @@ __device__ void sequence_draw(const GenericArgs& g, int b, const SeqRec& s, cons
         const int k = (s_found != 0x7fffffff) ? s_found : s_lastpos;
         g.t.out_tokens[(size_t)b * (g.t.gamma + 1) + s.n] = k;
         if (flag && g.t.out_status) g.t.out_status[b] |= flag;
-        g.ticket2[b] = 0u;
     }
 }
 

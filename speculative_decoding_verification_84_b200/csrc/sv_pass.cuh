@@ -1,34 +1,36 @@
 // sv_pass.cuh -- the streaming path for rows that are 16-byte aligned and at
-// least 4 KB: two persistent kernels.
+// least 4 KB: two kernels, the second a programmatic dependent of the first.
 //
-//   sv_pass1  the rows, in sequence order, form one stream of 16-byte vectors;
-//             warp w of the grid takes the contiguous span [w*S, (w+1)*S) and
-//             walks it on its own -- no barrier, no atomic -- 8 vectors per lane
-//             per batch, keeping per-lane online log-sum-exp state of l/T (the
-//             exponent arguments and sums on packed fp32 pairs) or the first
-//             argmax (T_b = 0).  Where its span crosses a row boundary (at most a
-//             few times) the warp reduces with shuffles and writes one Partial for
-//             that row segment.  A barrier per chunk would make every CTA wait for
-//             its slowest load; independent warps keep HBM busy.
-//             The warp whose segment holds a row's draft token x_j also stores
-//             the logit l[x_j] for the accept test.
-//   sv_pass2  one thread-block cluster per sequence b (clusters loop over the
-//             sequences): rank 0 finishes b -- fp64 combine of its partials,
-//             log-space accept scan [FlashSpec, Metodologia 1] (sequence_tail) --
-//             and a cluster barrier (hardware, no polling) hands the outcome to
-//             the cluster through distributed shared memory.  The cluster's CTAs
-//             then split the row pair the extra token is drawn from (residual
-//             max(0, p_n - q_n), or p_gamma for the bonus) [Speculative
-//             Speculative Decoding, Metodologia 2], each warp turning 32
-//             consecutive vectors (a tile) into one fp32 weight sum; after a
-//             second cluster barrier rank 0 draws the token by inverse CDF over
-//             b's tile sums.
-// Pass 1's grid holds as many CTAs as are resident at once (4 per SM at 256
-// threads and at most 64 registers), so every warp streams from start to end.
-// Pass 2 runs 2 CTAs per SM (the finish and the draw run in registers), in
-// clusters of up to 8 sized so that one wave covers the batch when it can; it is
-// launched as a programmatic dependent of pass 1: its CTAs start as pass-1 CTAs
-// leave and wait (griddepcontrol.wait) for all of pass 1 before reading.
+//   sv_stream  every warp of a resident grid takes one contiguous span of the
+//              row stream and walks it on its own (no barrier, no atomic, no
+//              wait), 4 vectors per lane per batch, keeping a lagging-offset
+//              log-sum-exp of l/T (sv_common.cuh) or the first argmax (T = 0).
+//              Where its span crosses a row boundary the warp reduces with
+//              shuffles and writes one Partial for that row segment; the warp
+//              holding a row's draft token keeps the logit l[x_j] for the accept
+//              test from its registers.  The next row's temperature and token are
+//              fetched one segment ahead, so no load waits on another.
+//              The rows are streamed by draft position, last position first and
+//              position 0 last: the rows a draw most often reads again (the
+//              first rejection is most often early) are the last ones streamed
+//              and are still in L2 when sv_draw reads them; rows streamed earlier
+//              are loaded with an L2 evict-first hint so they do not push them out.
+//   sv_draw    one thread-block cluster per sequence b (clusters loop over the
+//              sequences): rank 0 finishes b -- fp64 combine of the partials
+//              (every load of the finish in flight at once), the log-space
+//              accept test [FlashSpec, Metodologia 1] with the first rejection
+//              from one ballot -- and a cluster barrier hands the outcome to the
+//              cluster through distributed shared memory; the cluster's CTAs then
+//              split the draw rows (residual max(0, p_n - q_n), or p_gamma for
+//              the bonus token) [Speculative Speculative Decoding, Metodologia 2,
+//              "Conceito Central"; Desafios 2, "Amostragem Saguaro"] into tiles
+//              of 32 vectors, one fp32 weight sum per tile into rank 0's shared
+//              memory; after a second barrier rank 0 draws the token by inverse
+//              CDF over the tile sums.
+// sv_stream triggers its dependents at entry, so sv_draw's CTAs start as
+// sv_stream's leave; they fetch their sequence's inputs and then wait
+// (griddepcontrol.wait) for all of sv_stream before reading its partials.
+// Nothing is carried between calls: every slot a call reads, it wrote.
 #pragma once
 
 #include "sv_common.cuh"
@@ -40,25 +42,28 @@ namespace sv {
 
 namespace cg = cooperative_groups;
 
-constexpr int kPassThreads = 256;                  // = kThreads: reduce_lse / reduce_amax apply
-constexpr int kP1Vec = 8;                          // 16-byte vectors per lane per pass-1 batch
-constexpr int kMaxCluster = 8;                     // pass-2 cluster size limit (portable)
+constexpr int kPassThreads = 256;                  // = kThreads: block reductions apply
+constexpr int kStreamVec = 4;                      // 16-byte vectors per lane per sv_stream batch
+constexpr int kStreamSlots = 32;                   // partial slots per row (spans >= nq / 31 vectors)
+constexpr int kStreamSpanMin = 128;                // shortest span of a warp (vectors)
+constexpr int kMaxCluster = 8;                     // sv_draw cluster size limit (portable)
 constexpr int kTileSmem = 4096;                    // tile sums kept in rank 0's shared memory up to this many
 constexpr int kTileVecs = 32;                      // vectors per tile (one per lane)
+constexpr int kTileBatch = 8;                      // tiles per warp in flight in sv_draw
 constexpr int kStreamMinRowBytes = 4096;           // shorter rows take the generic path
 constexpr int kDrawQ = 16;                         // tile sums per lane per draw block
-constexpr int kSpanMin = 512;                      // shortest pass-1 span (vectors): bounds slots per row
 
 static_assert(kPassThreads == kThreads, "block reductions assume kThreads threads");
 
 struct PassArgs {
-    TailArgs t;              // t.nc = partial slots per row (stride and count); t.gath = gath
-    Partial* part;           // [B][R][t.nc]; the slots no span fills hold empty partials
-    float* gath;             // [B][2*gamma] the accept test's logits, written by pass 1
-    float* tsum;             // [B][NT2] weight sum of each tile
+    TailArgs t;              // t.nc = kStreamSlots
+    Partial* part;           // [B][R][kStreamSlots]; the slots no span fills hold empty partials
+    float* gath;             // [B][2*gamma] the accept test's logits, written by sv_stream
+    float* tsum;             // [B][NT2] weight sum of each tile (rows of more than kTileSmem tiles)
     const float* u_resample;
     long long nq;            // 16-byte vectors per row
-    long long S;             // vectors per warp span (pass 1)
+    long long S;             // vectors per warp span (sv_stream)
+    long long evict_rows;    // stream rows [0, evict_rows) load with an L2 evict-first hint
     int NT2;                 // tiles per row
     int B;
 };
@@ -79,41 +84,144 @@ __device__ __forceinline__ uint4 neg_inf_vec()
     return make_uint4(w, w, w, w);
 }
 
-// ----------------------------------------------------------------------------- pass 1
+// ----------------------------------------------------------------------------- sv_stream
 
-// One row segment [q0, q0 + n) of row (b, r) by one warp: batches of 32*kP1Vec
-// vectors (vector q0 + j*256 + u*32 + lane), reduced with shuffles; lane 0
-// writes the Partial.
+// Stream order of the rows: the bonus rows (target row gamma) of every sequence
+// first, then for j = gamma-1 down to 0 the pairs (target row j, draft row j) of
+// every sequence.  Stream row ro -> sequence b and row r of it (r > gamma: draft).
+__device__ __forceinline__ void stream_row(int gamma, int B, long long ro, int& b, int& r)
+{
+    if (ro < B) {
+        b = (int)ro;
+        r = gamma;
+        return;
+    }
+    const long long k = ro - B;
+    const int j = gamma - 1 - (int)(k / (2LL * B));
+    const long long m = k - (long long)(gamma - 1 - j) * 2LL * B;
+    b = (int)(m >> 1);
+    r = (m & 1) ? gamma + 1 + j : j;
+}
+
+// the draft position a row tests (-1 for the bonus row)
+__device__ __forceinline__ int row_position(int gamma, int r)
+{
+    return r < gamma ? r : (r > gamma ? r - gamma - 1 : -1);
+}
+
+template <bool EVF>
+__device__ __forceinline__ uint4 ld_row(const uint4* p, unsigned long long pol)
+{
+    if (!EVF) return ld_stream(p);
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// element e of a 16-byte vector
 template <int ESZ>
-__device__ __forceinline__ void pass1_segment(const PassArgs& g, int b, int r, long long q0, int n, Partial* dst)
+__device__ __forceinline__ float vec_elem(const uint4& v, int e)
+{
+    const int wi = ESZ == 2 ? (e >> 1) : e;
+    const unsigned w = wi == 0 ? v.x : (wi == 1 ? v.y : (wi == 2 ? v.z : v.w));
+    if (ESZ == 4) return __uint_as_float(w);
+    return (e & 1) ? bf16_hi(w) : bf16_lo(w);
+}
+
+// The exact form of a segment's sum, for a segment whose lagging offset was off
+// (sum outside [2^-40, 2^100), or not finite): the warp's maximum first, then the
+// sum of 2^(l*k - ceil(max*k_hi)).  Re-reads the segment (mostly from L2).
+template <int ESZ>
+__device__ __noinline__ float2 stream_exact(const uint4* p, int n, float khi, float klo, float mk)
+{
+    const int lane = threadIdx.x & 31;
+    float vm = -INFINITY;
+    for (int i = lane; i < n; i += 32) vm = fmaxf(vm, vec_max<ESZ>(ld_stream(p + i)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+    if (vm > -INFINITY && vm < INFINITY) mk = ceilf(__fmul_rn(vm, khi));
+    unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+    for (int i = lane; i < n; i += 32) {
+        const uint4 v = ld_stream(p + i);
+        lazy_exps_add<ESZ, 1>(acc, &v, khi, klo, mk);
+    }
+    return make_float2(mk, lazy_warp_sum(acc));
+}
+
+// One softmax segment [p, p + n) against the carried offset mk: the warp's
+// (offset, sum); *gval gets element ex of vector qx (qx < 0: none), in lane qx & 31.
+template <int ESZ, bool EVF>
+__device__ __forceinline__ float2 stream_softmax(const uint4* p, int n, float khi, float klo, float& mk, int qx,
+                                                 int ex, float* gval, unsigned long long pol)
+{
+    constexpr int CV = 32 * kStreamVec;
+    const int lane = threadIdx.x & 31;
+    const int kb = qx >= 0 ? qx / CV : -1;
+    const int ux = qx >= 0 ? (qx % CV) >> 5 : 0;
+    const int lx = qx & 31;
+    unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+    int jb = 0;
+    for (int j0 = 0; j0 < n; j0 += CV, ++jb) {
+        uint4 v[kStreamVec];
+        if (j0 + CV <= n) {
+#pragma unroll
+            for (int u = 0; u < kStreamVec; ++u) v[u] = ld_row<EVF>(p + j0 + u * 32 + lane, pol);
+        } else {
+#pragma unroll
+            for (int u = 0; u < kStreamVec; ++u) {
+                const int i = j0 + u * 32 + lane;
+                v[u] = i < n ? ld_row<EVF>(p + i, pol) : neg_inf_vec<ESZ>();
+            }
+        }
+        if (jb == kb && lane == lx) {
+            uint4 t = v[0];
+#pragma unroll
+            for (int u = 1; u < kStreamVec; ++u)
+                if (u == ux) t = v[u];
+            *gval = vec_elem<ESZ>(t, ex);
+        }
+        lazy_exps_add<ESZ, kStreamVec>(acc, v, khi, klo, mk);
+    }
+    const float s = lazy_warp_sum(acc);
+    if (s >= 0x1p-40f && s < 0x1p100f) return make_float2(mk, s);
+    const float2 r = stream_exact<ESZ>(p, n, khi, klo, mk);
+    mk = r.x;
+    return r;
+}
+
+// One row segment [q0, q0 + n) of row (b, r) with temperature T and draft token
+// x (-1 for the bonus row): the warp's Partial, and l[x] for the accept test.
+template <int ESZ>
+__device__ __forceinline__ void stream_segment(const PassArgs& g, int b, int r, float T, int x, long long q0, int n,
+                                               Partial* dst, float& mk, bool evf, unsigned long long pol)
 {
     constexpr int VEC = 16 / ESZ;
-    constexpr int kStep = 32 * kP1Vec;
+    constexpr int kStep = 32 * kStreamVec;
     const TailArgs& a = g.t;
     const int lane = threadIdx.x & 31;
-    const float T = __ldg(a.temperature + b);
-    const bool greedy = (T == 0.f);
-    if (!temperature_ok(T) || (greedy && r > a.gamma)) return;  // a row the finish will not read
+    if (!temperature_ok(T) || (T == 0.f && r > a.gamma)) return;  // a row the finish will not read
     const uint4* p = reinterpret_cast<const uint4*>(row_ptr<ESZ>(a, b, r)) + q0;
-    if (greedy) {
+    if (T == 0.f) {
         Amax A{-INFINITY, 0x7fffffff, 0};
         const int e0 = (int)(q0 * VEC);
         for (int j0 = 0; j0 < n; j0 += kStep) {
-            uint4 v[kP1Vec];
+            uint4 v[kStreamVec];
 #pragma unroll
-            for (int u = 0; u < kP1Vec; ++u) {
+            for (int u = 0; u < kStreamVec; ++u) {
                 const int i = j0 + u * 32 + lane;
                 v[u] = i < n ? ld_stream(p + i) : neg_inf_vec<ESZ>();
             }
 #pragma unroll
-            for (int u = 0; u < kP1Vec; ++u) {
-                float x[VEC];
-                unpack<ESZ>(v[u], x);
+            for (int u = 0; u < kStreamVec; ++u) {
+                float xv[VEC];
+                unpack<ESZ>(v[u], xv);
                 const int i0 = e0 + (j0 + u * 32 + lane) * VEC;
                 // fill elements (-inf past the segment) have larger indices than
                 // the real ones, so they never win a tie
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) amax_add(A, x[e], i0 + e);
+                for (int e = 0; e < VEC; ++e) amax_add(A, xv[e], i0 + e);
             }
         }
 #pragma unroll
@@ -124,77 +232,80 @@ __device__ __forceinline__ void pass1_segment(const PassArgs& g, int b, int r, l
             amax_merge(A, ob, oi, on);
         }
         if (lane == 0) *dst = Partial{A.best, 0.f, (float)A.nan, A.idx};
-    } else {
-        float khi, klo;
-        split_k(T, &khi, &klo);
-        Lse L;
-        lse_init(L);
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j0 = 0; j0 < n; j0 += kStep) {
-            uint4 v[kP1Vec];
-            if (j0 + kStep <= n) {
-#pragma unroll
-                for (int u = 0; u < kP1Vec; ++u) v[u] = ld_stream(p + j0 + u * 32 + lane);
-            } else {
-#pragma unroll
-                for (int u = 0; u < kP1Vec; ++u) {
-                    const int i = j0 + u * 32 + lane;
-                    v[u] = i < n ? ld_stream(p + i) : neg_inf_vec<ESZ>();  // -inf: weight 0
-                }
-            }
-            lse_group2<ESZ, kP1Vec>(L, acc, v, khi, klo);
+        return;
+    }
+    float khi, klo;
+    split_k(T, &khi, &klo);
+    int qx = -1, ex = 0;
+    if (x >= 0 && x < a.V) {
+        const long long q = (long long)(x / VEC) - q0;
+        if (q >= 0 && q < n) {
+            qx = (int)q;
+            ex = x % VEC;
         }
-        lse_fold(L, acc);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float om = __shfl_xor_sync(0xffffffffu, L.m, o);
-            const float omk = __shfl_xor_sync(0xffffffffu, L.mk, o);
-            const float os = __shfl_xor_sync(0xffffffffu, L.s, o);
-            lse_merge(L, om, omk, os);
-        }
-        if (lane == 0) {
-            *dst = Partial{L.m, L.mk, L.m == -INFINITY ? 0.f : L.s, 0};
-            // the accept test's logit l[x_j] of this row, if the segment holds it
-            // (target rows j < gamma and draft rows j; the bonus row has no token)
-            if (r != a.gamma) {
-                const int j = r < a.gamma ? r : r - a.gamma - 1;
-                const int x = __ldg(a.tokens + (size_t)b * a.gamma + j);
-                const long long e = (long long)x - q0 * VEC;
-                if (x >= 0 && x < a.V && e >= 0 && e < (long long)n * VEC)
-                    g.gath[(size_t)b * 2 * a.gamma + (r < a.gamma ? j : a.gamma + j)] =
-                        load_logit<ESZ>(p, (size_t)e);
-            }
-        }
+    }
+    float gval = 0.f;
+    const float2 ms = evf ? stream_softmax<ESZ, true>(p, n, khi, klo, mk, qx, ex, &gval, pol)
+                          : stream_softmax<ESZ, false>(p, n, khi, klo, mk, qx, ex, &gval, pol);
+    // an all -inf segment (sum 0) is an empty partial; m only marks presence
+    if (lane == 0) *dst = Partial{ms.y != 0.f ? 0.f : -INFINITY, ms.x, ms.y, 0};
+    if (qx >= 0 && lane == (qx & 31)) {
+        const int j = row_position(a.gamma, r);
+        g.gath[(size_t)b * 2 * a.gamma + (r < a.gamma ? j : a.gamma + j)] = gval;
     }
 }
 
 template <int ESZ>
-__global__ void __launch_bounds__(kPassThreads, 4) sv_pass1(PassArgs g)
+__global__ void __launch_bounds__(kPassThreads, 4) sv_stream(const __grid_constant__ PassArgs g)
 {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // sv_draw may be scheduled
     const TailArgs& a = g.t;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // pass 2 may be scheduled
+    const int lane = threadIdx.x & 31;
     const long long w = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
     const long long NQ = (long long)g.B * a.R * g.nq;
-    long long v0 = w * g.S;
-    const long long v1 = min(v0 + g.S, NQ);
-    while (v0 < v1) {
-        const long long row = v0 / g.nq;  // global row index b*R + r
-        const long long end = min(v1, (row + 1) * g.nq);
-        const int b = (int)(row / a.R), r = (int)(row - (long long)b * a.R);
-        // spans s0 .. w meet the row so far: this segment is its slot w - s0
-        const int slot = (int)(w - (row * g.nq) / g.S);
-        Partial* prow = g.part + (size_t)row * a.nc;
-        pass1_segment<ESZ>(g, b, r, v0 - row * g.nq, (int)(end - v0), prow + slot);
+    long long cur = w * g.S;
+    const long long v1 = min(cur + g.S, NQ);
+    if (cur >= v1) return;
+    unsigned long long pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    float mk = 0.f;  // lagging offset, carried across segments
+    long long ro = cur / g.nq;
+    int b, r;
+    stream_row(a.gamma, g.B, ro, b, r);
+    float T = __ldg(a.temperature + b);
+    int jp = row_position(a.gamma, r);
+    int x = jp >= 0 ? __ldg(a.tokens + (size_t)b * a.gamma + jp) : -1;
+    while (cur < v1) {
+        const long long rend = (ro + 1) * g.nq;
+        const long long pend = min(v1, rend);
+        // the next row's temperature and token, one segment ahead
+        int bn = 0, rn = 0, xn = -1;
+        float Tn = 0.f;
+        if (pend < v1) {
+            stream_row(a.gamma, g.B, ro + 1, bn, rn);
+            Tn = __ldg(a.temperature + bn);
+            const int jn = row_position(a.gamma, rn);
+            if (jn >= 0) xn = __ldg(a.tokens + (size_t)bn * a.gamma + jn);
+        }
+        // spans s0 .. w meet the row so far: this segment is slot w - s0
+        const int slot = (int)(w - (ro * g.nq) / g.S);
+        Partial* prow = g.part + ((size_t)b * a.R + r) * kStreamSlots;
+        stream_segment<ESZ>(g, b, r, T, x, cur - ro * g.nq, (int)(pend - cur), prow + slot, mk, ro < g.evict_rows,
+                            pol);
         // the span that ends the row marks the row's remaining slots empty, so the
-        // finish reads a fixed t.nc slots per row
-        const int lane = threadIdx.x & 31;
-        if (end == (row + 1) * g.nq)
-            for (int k = slot + 1 + lane; k < a.nc; k += 32) prow[k] = Partial{-INFINITY, 0.f, 0.f, 0x7fffffff};
-        v0 = end;
+        // finish reads a fixed kStreamSlots slots per row
+        if (pend == rend)
+            for (int k = slot + 1 + lane; k < kStreamSlots; k += 32) prow[k] = Partial{-INFINITY, 0.f, 0.f, 0x7fffffff};
+        cur = pend;
+        ++ro;
+        b = bn;
+        r = rn;
+        T = Tn;
+        x = xn;
     }
 }
 
-// ----------------------------------------------------------------------------- pass 2 and the draw
+// ----------------------------------------------------------------------------- sv_draw
 
 // A block of up to 32*kDrawQ tile sums: lane l holds tiles s0 + l*kDrawQ + q.
 struct TileBlock {
@@ -385,15 +496,14 @@ __device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& 
 }
 
 // Weight sums of tiles [k0, k1) of the row pair, one per warp-tile: warp w takes
-// tiles k0 + 8*(4j + u) + w (u < 4), lane l vector 32k + l, so each lane has 4
-// (or 8, with the draft row) loads in flight.  Vectors past the row read as -inf
-// target logits, whose weight is 0.
-template <int ESZ, bool PONLY>
+// tiles k0 + 8*(U*j + u) + w (u < U), lane l vector 32k + l, so each lane has U
+// (or 2U, with the draft row) loads in flight.  Vectors past the row read as
+// -inf target logits, whose weight is 0.
+template <int ESZ, bool PONLY, int U>
 __device__ void tile_range(const PassArgs& g, const SeqRec& rec, const uint4* tv, const uint4* dv, float* dst,
                            int k0, int k1)
 {
     constexpr int VEC = 16 / ESZ;
-    constexpr int U = 4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int kb = k0 + warp; kb < k1; kb += U * kWarps) {
         uint4 vt[U], vd[U];
@@ -422,19 +532,191 @@ __device__ void tile_range(const PassArgs& g, const SeqRec& rec, const uint4* tv
     }
 }
 
-template <int ESZ>
-__device__ __noinline__ void pass2_finish(const PassArgs& g, int b, TailSmem& ts, SeqRec* rec_out)
+
+// What the finish of one sequence needs from the inputs, fetched before
+// sv_draw waits for sv_stream (lane j < gamma of warp 0 holds position j).
+struct SeqIn {
+    float T;
+    int tok;
+    float ua;
+    float ur;
+};
+
+__device__ __forceinline__ SeqIn load_seq_in(const TailArgs& a, int b)
 {
+    const int tid = threadIdx.x;
+    SeqIn in;
+    in.T = __ldg(a.temperature + b);
+    in.tok = -1;
+    in.ua = 0.5f;
+    in.ur = 0.5f;
+    if (tid < a.gamma) {
+        in.tok = __ldg(a.tokens + (size_t)b * a.gamma + tid);
+        in.ua = __ldg(a.u_accept + (size_t)b * a.gamma + tid);
+    }
+    if (tid == 0) in.ur = __ldg(a.u_resample + b);
+    return in;
+}
+
+// Per-row results of the finish (shared memory of rank 0).
+struct FinishSmem {
+    double a2[kMaxRows];   // log2-normaliser of each row (NaN if bad)
+    double sum[kMaxRows];  // sum relative to the integer offset
+    float mk[kMaxRows];
+    int arg[kMaxRows];
+    int bad[kMaxRows];
+    float gath[2 * SV_MAX_GAMMA];
+    int status, n;
+};
+
+// Finish sequence b with one CTA: warp w folds rows w, w + 8, ... (lane l reads
+// slot l of each, every load in flight at once) in fp64; gathers log p_j(x_j)
+// and log q_j(x_j) [FlashSpec, Metodologia 1, "Mecanismo"]; warp 0 runs the
+// log-space test at every draft position and takes the first rejection from one
+// ballot; writes the accepted prefix, -1 padding, n_accepted, status and
+// normalisers, and the draw record into *rec_out.
+template <int ESZ>
+__device__ __noinline__ void finish_cta(const PassArgs& g, int b, const SeqIn& in, FinishSmem& fs, SeqRec* rec_out)
+{
+    constexpr int kRowIter = (kMaxRows + kWarps - 1) / kWarps;
     const TailArgs& a = g.t;
-    sequence_tail<ESZ, kPassThreads, BlockSync>(a, b, threadIdx.x, FloatPartials{a.part}, ts);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gamma = a.gamma, R = a.R;
+    const float T = in.T;
+    const bool greedy = (T == 0.f);
+    const bool tval = temperature_ok(T);
+    const int rows_used = !tval ? 0 : (greedy ? gamma + 1 : R);
+
+    const float4* pp = reinterpret_cast<const float4*>(g.part) + (size_t)b * R * kStreamSlots;
+    const float4 kEmpty = make_float4(-INFINITY, 0.f, 0.f, __int_as_float(0x7fffffff));
+    float4 q[kRowIter];
+#pragma unroll
+    for (int k = 0; k < kRowIter; ++k) {
+        const int r = warp + kWarps * k;
+        q[k] = r < rows_used ? __ldcg(pp + (size_t)r * kStreamSlots + lane) : kEmpty;
+    }
+    if (tid < 2 * gamma && tval && !greedy) fs.gath[tid] = __ldcg(g.gath + (size_t)b * 2 * gamma + tid);
+#pragma unroll
+    for (int k = 0; k < kRowIter; ++k) {
+        const int r = warp + kWarps * k;
+        if (r >= rows_used) break;
+        if (greedy) {
+            Amax A{q[k].x, __float_as_int(q[k].w), q[k].z != 0.f};
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ob = __shfl_xor_sync(0xffffffffu, A.best, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, A.idx, o);
+                const int on = __shfl_xor_sync(0xffffffffu, A.nan, o);
+                amax_merge(A, ob, oi, on);
+            }
+            if (lane == 0) {
+                fs.arg[r] = A.idx;
+                fs.bad[r] = A.nan || A.best == INFINITY || A.best == -INFINITY;
+            }
+        } else {
+            const bool has = (q[k].x != -INFINITY);
+            float MK = has ? q[k].y : -INFINITY;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) MK = fmaxf(MK, __shfl_xor_sync(0xffffffffu, MK, o));
+            double S = has ? (double)q[k].z * pow2d(q[k].y - MK) : 0.0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+            if (lane == 0) {
+                const bool bad = (MK == -INFINITY) || !isfinite(S) || !(S > 0.0);
+                fs.bad[r] = bad;
+                fs.mk[r] = MK;
+                fs.sum[r] = S;
+                fs.a2[r] = bad ? (double)NAN : (double)MK + log2(S);
+            }
+        }
+    }
     __syncthreads();
-    if (threadIdx.x == 0) *rec_out = ts.rec;
+
+    if (warp == 0) {
+        int st = 0;
+        const int x_j = (lane < gamma) ? in.tok : -1;
+        if (!tval) {
+            st = SV_ROW_BAD_TEMPERATURE;
+        } else {
+            const int badtok = (lane < gamma) && (x_j < 0 || x_j >= a.V);
+            int badrow = 0;
+            for (int r = lane; r < rows_used; r += 32) badrow |= fs.bad[r];
+            // the uniforms stand for draws of U[0, 1): anything else (NaN included)
+            // is an invalid input (a greedy sequence reads none)
+            int bad_u = 0;
+            if (!greedy) {
+                if (lane < gamma) bad_u = !(in.ua >= 0.f && in.ua < 1.f);
+                if (lane == 0) bad_u |= !(in.ur >= 0.f && in.ur < 1.f);
+            }
+            if (__any_sync(0xffffffffu, badtok)) st |= SV_ROW_BAD_TOKEN;
+            if (__any_sync(0xffffffffu, badrow)) st |= SV_ROW_BAD_LOGITS;
+            if (__any_sync(0xffffffffu, bad_u)) st |= SV_ROW_BAD_UNIFORM;
+        }
+        bool acc = false;
+        if (st == 0 && lane < gamma) {
+            if (greedy) {
+                acc = (x_j == fs.arg[lane]);
+            } else {
+                const double Td = (double)T;
+                const double lp = (double)fs.gath[lane] / Td - fs.a2[lane] * kLn2;
+                const double lq = (double)fs.gath[gamma + lane] / Td - fs.a2[gamma + 1 + lane] * kLn2;
+                acc = log((double)in.ua) < (lp - lq);
+            }
+        }
+        const unsigned mask = (gamma == 32) ? 0xffffffffu : ((1u << gamma) - 1u);
+        const unsigned rej = __ballot_sync(0xffffffffu, !acc) & mask;
+        const int n = (st != 0) ? 0 : (rej ? __ffs(rej) - 1 : gamma);
+        if (lane == 0) {
+            fs.status = st;
+            fs.n = n;
+        }
+    }
+    __syncthreads();
+
+    const int st = fs.status, n = fs.n;
+    int32_t* ot = a.out_tokens + (size_t)b * (gamma + 1);
+    for (int j = tid; j <= gamma; j += kPassThreads) {
+        int v = -1;
+        if (st == 0) {
+            if (j < n) v = __ldg(a.tokens + (size_t)b * gamma + j);
+            else if (j == n && greedy) v = fs.arg[n];
+        }
+        ot[j] = v;  // a sampled extra token is written by the draw
+    }
+    if (a.out_log_norm) {
+        double* ln = a.out_log_norm + (size_t)b * R;
+        for (int r = tid; r < R; r += kPassThreads)
+            ln[r] = (tval && !greedy && !fs.bad[r]) ? fs.a2[r] * kLn2 : (double)NAN;
+    }
+    if (tid == 0) {
+        a.out_n[b] = n;
+        if (a.out_status) a.out_status[b] = st;
+        SeqRec rec;
+        rec.mode = (st != 0 || greedy) ? kModeNone : (n < gamma ? kModeResidual : kModeBonus);
+        rec.n = n;
+        rec.mk_t = 0.f;
+        rec.inv_s_t = 0.f;
+        rec.mk_d = 0.f;
+        rec.inv_s_d = 0.f;
+        rec.k_hi = 0.f;
+        rec.k_lo = 0.f;
+        if (rec.mode != kModeNone) {
+            split_k(T, &rec.k_hi, &rec.k_lo);
+            rec.mk_t = fs.mk[n];
+            rec.inv_s_t = (float)(1.0 / fs.sum[n]);
+            if (rec.mode == kModeResidual) {
+                rec.mk_d = fs.mk[gamma + 1 + n];
+                rec.inv_s_d = (float)(1.0 / fs.sum[gamma + 1 + n]);
+            }
+        }
+        *rec_out = rec;
+    }
 }
 
 template <int ESZ>
-__global__ void __launch_bounds__(kPassThreads, 2) sv_pass2(PassArgs g)
+__global__ void __launch_bounds__(kPassThreads, 2) sv_draw(const __grid_constant__ PassArgs g)
 {
-    __shared__ TailSmem s_tail;
+    __shared__ FinishSmem s_fin;
     __shared__ SeqRec s_rec;
     __shared__ float s_tiles[kTileSmem];  // rank 0: b's tile sums, written by the whole cluster
     cg::cluster_group cluster = cg::this_cluster();
@@ -444,12 +726,14 @@ __global__ void __launch_bounds__(kPassThreads, 2) sv_pass2(PassArgs g)
     const bool tiles_in_smem = g.NT2 <= kTileSmem;
     float* tiles0 = cluster.map_shared_rank(s_tiles, 0);  // rank 0's buffer, from any rank
 
-    // wait until pass 1 has completed and its writes are visible (a no-op when
-    // this launch did not overlap pass 1)
+    // the first sequence's inputs are not sv_stream's outputs: fetch them before
+    // waiting for sv_stream to complete and its writes to be visible
+    SeqIn in = cid < g.B ? load_seq_in(t, cid) : SeqIn{0.f, -1, 0.5f, 0.5f};
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     for (int b = cid; b < g.B; b += nclusters) {
-        if (rank == 0) pass2_finish<ESZ>(g, b, s_tail, &s_rec);
+        if (b != cid) in = load_seq_in(t, b);
+        if (rank == 0) finish_cta<ESZ>(g, b, in, s_fin, &s_rec);
         cluster.sync();  // rank 0's outcome is visible to the cluster
         const SeqRec rec = *cluster.map_shared_rank(&s_rec, 0);
         float* dst = tiles_in_smem ? tiles0 : g.tsum + (size_t)b * g.NT2;
@@ -460,8 +744,8 @@ __global__ void __launch_bounds__(kPassThreads, 2) sv_pass2(PassArgs g)
             // this CTA's share of the tiles
             const int per = (g.NT2 + cs - 1) / cs;
             const int k0 = rank * per, k1 = min(g.NT2, k0 + per);
-            if (bonus) tile_range<ESZ, true>(g, rec, tv, tv, dst, k0, k1);
-            else tile_range<ESZ, false>(g, rec, tv, dv, dst, k0, k1);
+            if (bonus) tile_range<ESZ, true, kTileBatch>(g, rec, tv, tv, dst, k0, k1);
+            else tile_range<ESZ, false, kTileBatch>(g, rec, tv, dv, dst, k0, k1);
         }
         cluster.sync();  // every tile sum of b is visible to rank 0
         if (rank == 0 && rec.mode != kModeNone) pass2_draw<ESZ>(g, b, rec, tiles_in_smem ? s_tiles : dst, tiles_in_smem);

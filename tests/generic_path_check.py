@@ -17,7 +17,7 @@ from speculative_decoding_verification_84_b200 import binding, workloads as W  #
 def main():
     assert os.environ.get("SPEC_VERIFY_FORCE_GENERIC") == "1"
     import torch
-    assert binding.kernels_per_call(64, 5, 128256, torch.bfloat16) == 2
+    assert binding.kernels_per_call(64, 5, 128256, torch.bfloat16) == 3
     cases = [W.make_workload("c2"), W.make_workload("c3", seqs=range(16)),
              W.make_random(9, 3, 8192, "bf16", seed=77, T=np.array([0.0, 0.7, 1.0] * 3, np.float32))]
     for w in cases:

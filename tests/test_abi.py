@@ -54,9 +54,10 @@ def test_workspace_size_host_only(lib):
     assert lib.spec_verify_workspace_size(4, 33, 100, 0) == 0
     assert lib.spec_verify_workspace_size(4, 2, 0, 0) == 0
     assert lib.spec_verify_workspace_size(4, 2, 100, 7) == 0
-    # two launches per call for either kernel family (aligned 4 KB+ rows or not), 0 on a bad shape
+    # two launches per call on 16-byte-aligned rows of 4 KB or more (stream, draw), three
+    # otherwise (ticket reset, row pass, resample), 0 on a bad shape
     assert lib.spec_verify_kernels_per_call(64, 5, 128256, 1) == 2
-    assert lib.spec_verify_kernels_per_call(3, 2, 3001, 1) == 2
+    assert lib.spec_verify_kernels_per_call(3, 2, 3001, 1) == 3
     assert lib.spec_verify_kernels_per_call(0, 2, 100, 0) == 0
     # a larger batch never needs less workspace
     sizes = [lib.spec_verify_workspace_size(b, 5, 128256, 1) for b in (1, 2, 64, 65, 256)]
