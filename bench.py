@@ -4,7 +4,10 @@ One step = one spec_verify call (every kernel of the path) over one batch of the
 workload "c3": B=64 sequences, gamma=5, V=128256, bf16 logits (Zipf-biased
 N(0,3^2) target, rho=0.9 draft, T=1).  Inputs are resident in HBM before the
 timed region; calls rotate over several copies of the batch so that every call
-reads logits last touched > 2x L2 (126 MB) earlier.
+reads logits last touched > 2x L2 (126 MB) earlier.  At least 200 ms of untimed
+calls run first, so the timed calls start at steady clocks.  After the timed
+region the line also gets ``per_config``: the same numbers for all five
+workloads (c1..c5; c1 and c2 also with their logits hot in L2).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -169,6 +172,109 @@ def run_reference(args):
     return 0
 
 
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (context for the measured copy peak)
+PER_CONFIG = ("c1", "c2", "c3", "c4", "c5")
+L2_BYTES = 126 * 2 ** 20
+
+
+class Caller:
+    """One workload resident on the device, rotated over enough copies that each
+    call reads logits last touched more than 2x L2 earlier (cold), or one copy
+    reused (hot), with its outputs and workspace; call(i) verifies copy i."""
+
+    def __init__(self, w, dev, lib, binding, hot=False):
+        import torch
+        self.w, self.lib, self.binding = w, lib, binding
+        self.B, self.gamma, self.V = w.B, w.gamma, w.V
+        self.esz = 2 if w.dtype == "bf16" else 4
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.base = binding.to_device(w, dev)
+        self.n_copies = 1 if hot else max(3, int(np.ceil(2 * L2_BYTES / w.logits_bytes())) + 1)
+        self.sets = [self.base] + [{k: v.clone() for k, v in self.base.items()} for _ in range(self.n_copies - 1)]
+        self.out_t = torch.empty((w.B, w.gamma + 1), dtype=torch.int32, device=dev)
+        self.out_n = torch.empty((w.B,), dtype=torch.int32, device=dev)
+        self.wsz = binding.workspace_size(w.B, w.gamma, w.V, tdt)
+        self.wspace = torch.empty(self.wsz, dtype=torch.uint8, device=dev)  # needs no initialisation
+        self.stream = torch.cuda.current_stream(dev)
+        self.dt_code = binding._dt_code(tdt)
+        self.kernels_per_call = binding.kernels_per_call(w.B, w.gamma, w.V, tdt)
+        self.alg = algorithmic_bytes(w.B, w.gamma, w.V, self.esz)
+
+    def call(self, i, d=None):
+        d = self.sets[i % self.n_copies] if d is None else d
+        st = self.lib.spec_verify(d["target"].data_ptr(), d["draft"].data_ptr(), self.dt_code,
+                                  d["draft_tokens"].data_ptr(), d["temperature"].data_ptr(),
+                                  d["u_accept"].data_ptr(), d["u_resample"].data_ptr(), self.out_t.data_ptr(),
+                                  self.out_n.data_ptr(), self.B, self.gamma, self.V, self.wspace.data_ptr(),
+                                  self.wsz, None, None, self.stream.cuda_stream)
+        if st != 0:
+            raise RuntimeError(self.binding.status_string(st))
+
+    def prewarm(self, seconds):
+        """Untimed back-to-back calls for about `seconds`, so timing starts at steady clocks."""
+        import torch
+        self.call(0)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        i = 1
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(64):
+                self.call(i)
+                i += 1
+            torch.cuda.synchronize()
+
+    def time_back_to_back(self, k):
+        """Mean ms per call of k calls bracketed by two events on the launching stream
+        (an event between calls would add its own gap to every call)."""
+        import torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(self.stream)
+        for i in range(k):
+            self.call(i)
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / k
+
+    def single_calls(self, k):
+        """ms of k single calls, each between its own event pair."""
+        import torch
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * k)]
+        for i in range(k):
+            ev[2 * i].record(self.stream)
+            self.call(i)
+            ev[2 * i + 1].record(self.stream)
+        torch.cuda.synchronize()
+        return [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(k)]
+
+
+def config_line(c, peak, peak_kind, hot=False, budget_ms=20.0):
+    """Per-workload numbers: mean (back to back) and single-call spread, seq-steps/s,
+    algorithmic bytes per call and the fractions of the HBM peak (measured copy
+    bandwidth when available, else the fallback figure; ``peak_source`` says which)
+    and of the nominal 8 TB/s."""
+    c.prewarm(0.05)
+    probe = c.time_back_to_back(8)
+    k = int(max(20, min(4000, budget_ms / max(probe, 1e-4))))
+    mean_ms = c.time_back_to_back(k)
+    sc = c.single_calls(min(k, 200))
+    gbs = c.alg / (mean_ms / 1e3) / 1e9
+    return {
+        "workload": c.w.name, "B": c.B, "gamma": c.gamma, "V": c.V, "dtype": c.w.dtype,
+        "kernels_per_call": c.kernels_per_call, "calls_timed": k,
+        "us_per_call_mean": 1e3 * mean_ms,
+        "us_single_call_p10": 1e3 * float(np.percentile(sc, 10)),
+        "us_single_call_p50": 1e3 * float(np.percentile(sc, 50)),
+        "us_single_call_p90": 1e3 * float(np.percentile(sc, 90)),
+        "seq_steps_per_s": c.B / (mean_ms / 1e3),
+        "algorithmic_bytes": c.alg, "hbm_gbs": gbs,
+        "frac_of_peak": gbs / peak, "peak_gbs": peak, "peak_source": peak_kind,
+        "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS,
+        "l2": ("hot: one copy reused" if hot else
+               f"cold: {c.n_copies} copies rotated ({c.n_copies * c.w.logits_bytes() / 1e6:.0f} MB)"),
+    }
+
+
 def run_ours(args):
     import torch
     ws, rank, local = dist_env()
@@ -186,51 +292,31 @@ def run_ours(args):
     lib = binding.load_library()
 
     w = W.make_workload(WORKLOAD)
-    B, gamma, V = w.B, w.gamma, w.V
-    esz = 2 if w.dtype == "bf16" else 4
-    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    base = binding.to_device(w, dev)
-    l2_bytes = 126 * 2 ** 20
-    n_copies = max(3, int(np.ceil(2 * l2_bytes / w.logits_bytes())) + 1)
-    sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_copies - 1)]
-    out_t = torch.empty((B, gamma + 1), dtype=torch.int32, device=dev)
-    out_n = torch.empty((B,), dtype=torch.int32, device=dev)
-    wsz = binding.workspace_size(B, gamma, V, tdt)
-    wspace = torch.zeros(wsz, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    dt_code = binding._dt_code(tdt)
-    kernels_per_call = binding.kernels_per_call(B, gamma, V, tdt)
-    rowbytes = V * esz
-    kernel_name = ("sv_stream + sv_draw (one call; sv_stream reads every logit once)"
-                   if rowbytes % 16 == 0 and rowbytes >= 4096 else "sv_reset + sv_rowpass + sv_resample (one call)")
-
-    def call(d):
-        st = lib.spec_verify(d["target"].data_ptr(), d["draft"].data_ptr(), dt_code, d["draft_tokens"].data_ptr(),
-                             d["temperature"].data_ptr(), d["u_accept"].data_ptr(), d["u_resample"].data_ptr(),
-                             out_t.data_ptr(), out_n.data_ptr(), B, gamma, V, wspace.data_ptr(), wsz, None, None,
-                             stream.cuda_stream)
-        if st != 0:
-            raise RuntimeError(binding.status_string(st))
+    c = Caller(w, dev, lib, binding)
+    B, gamma, V, esz = c.B, c.gamma, c.V, c.esz
+    kernel_name = {1: "sv_small (one call: one warp per sequence)",
+                   2: "sv_stream + sv_draw (one call; sv_stream reads every logit once)",
+                   3: "sv_reset + sv_rowpass + sv_resample (one call)"}[c.kernels_per_call]
 
     def barrier():
         if pg is not None:
             pg.barrier()
 
     for i in range(max(3, args.warmup)):
-        call(sets[i % n_copies])
+        c.call(i)
     torch.cuda.synchronize()
+    c.prewarm(0.25)  # >= 200 ms of back-to-back calls: the timed calls start at steady clocks
 
-    # timed region: K back-to-back calls bracketed by two events on the launching
-    # stream (an event between calls would add its own gap to every call)
+    # timed region: K back-to-back calls bracketed by two events on the launching stream
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     sampler.start()
     barrier()
     torch.cuda.synchronize()
-    e_start.record(stream)
+    e_start.record(c.stream)
     for i in range(args.steps):
-        call(sets[i % n_copies])
-    e_end.record(stream)
+        c.call(i)
+    e_end.record(c.stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
@@ -238,31 +324,23 @@ def run_ours(args):
     value, total_ms = job_value(local_ms, ws, B * args.steps, pg, dev)
     ms_per_step = total_ms / args.steps
 
-    # spread of single calls, from a separate untimed sample with an event pair
-    # around each call
-    n_spread = min(args.steps, 200)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_spread)]
-    for i in range(n_spread):
-        ev[2 * i].record(stream)
-        call(sets[i % n_copies])
-        ev[2 * i + 1].record(stream)
-    torch.cuda.synchronize()
-    per_call = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n_spread)]
+    # spread of single calls, from a separate untimed sample with an event pair around each
+    per_call = c.single_calls(min(args.steps, 200))
 
-    alg = algorithmic_bytes(B, gamma, V, esz)
+    alg = c.alg
     mean_call_ms = local_ms / args.steps  # this rank's mean call over the timed region
     achieved = alg / (mean_call_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
 
     # end to end through the public API: pinned host inputs -> device, call, outputs -> host
     host = {}
-    for k, v in base.items():
+    for k, v in c.base.items():
         h = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
         h.copy_(v)
         host[k] = h
     h_out_t = torch.empty((B, gamma + 1), dtype=torch.int32, pin_memory=True)
     h_out_n = torch.empty((B,), dtype=torch.int32, pin_memory=True)
-    dbuf = {k: torch.empty_like(v) for k, v in base.items()}
+    dbuf = {k: torch.empty_like(v) for k, v in c.base.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = h_out_t.numel() * 4 + h_out_n.numel() * 4
     e2e_steps = max(3, min(args.steps, 50))
@@ -270,21 +348,43 @@ def run_ours(args):
     def e2e_step():
         for k in dbuf:
             dbuf[k].copy_(host[k], non_blocking=True)
-        call(dbuf)
-        h_out_t.copy_(out_t, non_blocking=True)
-        h_out_n.copy_(out_n, non_blocking=True)
+        c.call(0, dbuf)
+        h_out_t.copy_(c.out_t, non_blocking=True)
+        h_out_n.copy_(c.out_n, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(c.stream)
     for _ in range(e2e_steps):
         e2e_step()
-    e1.record(stream)
+    e1.record(c.stream)
     torch.cuda.synchronize()
     e2e_value, _ = job_value(e0.elapsed_time(e1), ws, B * e2e_steps, pg, dev)
+    del dbuf, host
+
+    # every workload on this GPU (rank 0 at N = 1): not part of the timed region above
+    per_config = None
+    if rank == 0 and ws == 1 and not args.no_per_config:
+        per_config = {"c3": config_line(c, peak, peak_kind)}
+        del c
+        for name in PER_CONFIG:
+            if name == WORKLOAD:
+                continue
+            wc = W.make_workload(name)
+            cc = Caller(wc, dev, lib, binding)
+            per_config[name] = config_line(cc, peak, peak_kind)
+            if name in ("c1", "c2"):  # latency-bound: also with the logits hot in L2
+                del cc
+                ch = Caller(wc, dev, lib, binding, hot=True)
+                per_config[name + "_hot_l2"] = config_line(ch, peak, peak_kind, hot=True)
+                del ch
+            else:
+                del cc
+            del wc
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -311,10 +411,13 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD_DESC, "global_batch": ws * B, "gamma": gamma, "V": V,
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                   "l2": f"inputs rotate over {n_copies} resident copies ({n_copies * w.logits_bytes() / 1e6:.0f} MB > 2x L2)"},
+                   "l2": f"inputs rotate over {c_copies(w)} resident copies "
+                         f"({c_copies(w) * w.logits_bytes() / 1e6:.0f} MB > 2x L2)"},
         "hbm_gbs": achieved, "pct_of_peak": 100.0 * achieved / peak,
+        "pct_of_nominal_8tbs": 100.0 * achieved / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "kernel": kernel_name,
                      "algorithmic_bytes_per_launch": alg, "mean_launch_us": 1e3 * mean_call_ms,
                      "single_call_p10_us": 1e3 * float(np.percentile(per_call, 10)),
@@ -322,11 +425,16 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "seq-steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": kernels_per_call * args.steps,
+        "gpu_launches": binding.kernels_per_call(B, gamma, V, torch.bfloat16) * args.steps,
         "clocks": clocks,
+        "per_config": per_config,
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def c_copies(w):
+    return max(3, int(np.ceil(2 * L2_BYTES / w.logits_bytes())) + 1)
 
 
 def main():
@@ -337,6 +445,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the line's per-workload numbers")
     args = ap.parse_args()
     if args.impl == "reference":
         if args.steps > 200:

@@ -99,9 +99,11 @@ typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
  */
 size_t spec_verify_workspace_size(int B, int gamma, int V, sv_dtype dt);
 
-/* Number of kernel launches one spec_verify() call of this shape enqueues (3:
- * the counter reset, then one streaming kernel or two general kernels), or 0 on
- * a bad shape.  Infrastructure: no passage of the pages stands behind it. */
+/* Number of kernel launches one spec_verify() call of this shape enqueues: 1
+ * for rows of at most 256 elements (one warp per sequence), 2 for 16-byte-aligned
+ * rows of at least 4 KB (the streaming pass, then the draw), 3 otherwise (ticket
+ * reset, row pass, resample); 0 on a bad shape.  Infrastructure: no passage of
+ * the pages stands behind it. */
 int spec_verify_kernels_per_call(int B, int gamma, int V, sv_dtype dt);
 
 /* cudaMemsetAsync(workspace, 0, workspace_bytes, stream).  Not required before

@@ -7,9 +7,11 @@
 //     sequence, sums its draw rows (mostly from L2) and draws.  Used when every
 //     row is 16-byte aligned (V * element size a multiple of 16) and at least
 //     4 KB long.  Every slot these kernels read, the same call wrote.
-//   * sv_reset + sv_rowpass + sv_resample (sv_generic.cuh): any shape; sv_reset
-//     zeroes the per-sequence tickets first, so a workspace carries nothing from
-//     one call to the next.
+//   * sv_small (sv_small.cuh): rows of at most kSmallMaxV elements; one warp per
+//     sequence with the rows in registers, one launch, no workspace traffic.
+//   * sv_reset + sv_rowpass + sv_resample (sv_generic.cuh): any other shape;
+//     sv_reset zeroes the per-sequence tickets first, so a workspace carries
+//     nothing from one call to the next.
 // SPEC_VERIFY_FORCE_GENERIC=1 in the environment selects the second family for
 // every shape (both compute the same results; tests use it to cover both).
 #include "spec_verify.h"
@@ -25,6 +27,7 @@
 #include "sv_common.cuh"
 #include "sv_generic.cuh"
 #include "sv_pass.cuh"
+#include "sv_small.cuh"
 
 namespace {
 
@@ -42,7 +45,7 @@ constexpr long long kL2KeepBytes = 80LL << 20;
 
 struct Plan {
     int B, gamma, V, R, esz;
-    bool stream;
+    bool small, stream;
     int nc1, C1, nc2, C2;           // generic
     int nslot, NT2;                 // stream
     long long evict_rows;           // stream: rows loaded evict-first
@@ -77,6 +80,7 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     p->esz = dt == SV_DTYPE_BF16 ? 2 : 4;
     p->rowbytes = (long long)V * p->esz;
     const long long rows = (long long)B * p->R;
+    p->small = !force_generic() && V <= kSmallMaxV;
     p->stream = !force_generic() && (p->rowbytes % 16 == 0) && (p->rowbytes >= kStreamMinRowBytes);
 
     // generic split: ~32 KB per CTA, but at least ~2 CTAs per SM in total
@@ -121,7 +125,7 @@ bool make_plan(int B, int gamma, int V, sv_dtype dt, Plan* p)
     off = align256(off + sizeof(Partial) * (size_t)nparts);
     p->off_rsum = off;
     off = align256(off + sizeof(double) * (size_t)nrsum);
-    p->total = off;
+    p->total = p->small ? 256 : off;  // the small path keeps everything in registers
     return true;
 }
 
@@ -146,7 +150,7 @@ template <class K>
 int ctas_per_sm(K kernel, int slot)
 {
     static std::mutex mu;
-    static int cache[4][kMaxDevices] = {};
+    static int cache[32][kMaxDevices] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
     std::lock_guard<std::mutex> lock(mu);
@@ -186,6 +190,37 @@ int max_clusters(int cs)
     return cache[cs][dev];
 }
 
+template <int ESZ, int G, int E>
+cudaError_t launch_small_ge(const TailArgs& t, int B, cudaStream_t st)
+{
+    constexpr int slot = 2 + (G == 8 ? 0 : (G == 16 ? 4 : 8)) + (E == 1 ? 0 : (E == 2 ? 1 : (E == 4 ? 2 : 3)));
+    const int c = ctas_per_sm(sv_small<ESZ, G, E>, slot + (ESZ == 4 ? 12 : 0));
+    if (c < 1) return cudaErrorInvalidConfiguration;
+    const long long seqs_per_cta = (long long)kWarps * (32 / G);
+    const long long grid = std::min<long long>((long long)c * device_sm_count(), cdiv(B, seqs_per_cta));
+    sv_small<ESZ, G, E><<<(unsigned)grid, kThreads, 0, st>>>(t, B);
+    return cudaGetLastError();
+}
+
+template <int ESZ, int G>
+cudaError_t launch_small_g(int E, const TailArgs& t, int B, cudaStream_t st)
+{
+    switch (E) {
+    case 1: return launch_small_ge<ESZ, G, 1>(t, B, st);
+    case 2: return launch_small_ge<ESZ, G, 2>(t, B, st);
+    case 4: return launch_small_ge<ESZ, G, 4>(t, B, st);
+    default: return launch_small_ge<ESZ, G, 8>(t, B, st);
+    }
+}
+
+template <int ESZ>
+cudaError_t launch_small(int G, int E, const TailArgs& t, int B, cudaStream_t st)
+{
+    if (G == 8) return launch_small_g<ESZ, 8>(E, t, B, st);
+    if (G == 16) return launch_small_g<ESZ, 16>(E, t, B, st);
+    return launch_small_g<ESZ, 32>(E, t, B, st);
+}
+
 template <int ESZ>
 cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_t* tokens,
                    const float* temperature, const float* u_acc, const float* u_res, int32_t* out_tokens,
@@ -209,6 +244,15 @@ cudaError_t launch(const Plan& p, const void* tgt, const void* dft, const int32_
     t.gamma = p.gamma;
     t.V = p.V;
     t.R = p.R;
+
+    if (p.small) {
+        // groups of G lanes per sequence (the smallest of 8, 16, 32 with G >= gamma
+        // and 8 * G >= V), E elements of a row per lane
+        const int G = (p.gamma <= 8 && p.V <= 64) ? 8 : ((p.gamma <= 16 && p.V <= 128) ? 16 : 32);
+        const int per = (int)cdiv(p.V, G);
+        const int E = per <= 1 ? 1 : (per <= 2 ? 2 : (per <= 4 ? 4 : 8));
+        return launch_small<ESZ>(G, E, t, p.B, st);
+    }
 
     if (p.stream) {
         PassArgs g;
@@ -317,7 +361,8 @@ extern "C" int spec_verify_kernels_per_call(int B, int gamma, int V, sv_dtype dt
 {
     Plan p;
     if (!make_plan(B, gamma, V, dt, &p)) return 0;
-    return p.stream ? 2 : 3;  // sv_stream + sv_draw, or sv_reset + sv_rowpass + sv_resample
+    // sv_small; sv_stream + sv_draw; or sv_reset + sv_rowpass + sv_resample
+    return p.small ? 1 : (p.stream ? 2 : 3);
 }
 
 extern "C" sv_status spec_verify_workspace_init(void* workspace, size_t workspace_bytes,

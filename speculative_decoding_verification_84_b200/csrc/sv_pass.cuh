@@ -324,11 +324,15 @@ __device__ __forceinline__ void load_tile_block(TileBlock& tb, const float* w, i
         const int idx = s0 + lane * kDrawQ + q;
         tb.v[q] = idx < n ? (smem ? w[idx] : __ldcg(w + idx)) : 0.f;
     }
-    double s = 0.0;
+    double t[kDrawQ / 2];
 #pragma unroll
-    for (int q = 0; q < kDrawQ; ++q) s += (double)tb.v[q];
-    tb.ls = s;
-    tb.incl = warp_inclusive_scan(s);
+    for (int q = 0; q < kDrawQ / 2; ++q) t[q] = (double)tb.v[2 * q] + (double)tb.v[2 * q + 1];
+#pragma unroll
+    for (int w = kDrawQ / 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int q = 0; q < w; ++q) t[q] += t[q + w];
+    tb.ls = t[0];
+    tb.incl = warp_inclusive_scan(tb.ls);
 }
 
 // First tile of the block whose running sum (from `carry`) exceeds target, or -1;
@@ -454,7 +458,7 @@ __device__ void tile_sums_strided(const PassArgs& g, const SeqRec& rec, bool p_o
 // smallest token k with C_k > u * S over b's tile sums; a vanished residual
 // (S = 0) falls back to p_n, whose tile sums the CTA computes first.
 template <int ESZ>
-__device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& rec, float* ws, bool smem)
+__device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& rec, float* ws, bool smem, float ur)
 {
     __shared__ double s_S;
     const TailArgs& t = g.t;
@@ -463,8 +467,11 @@ __device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& 
     const bool bonus = (rec.mode == kModeBonus);
     const uint4* tv = reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, rec.n));
     const uint4* dv = bonus ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
+    // warp 0 keeps the first block of tile sums in registers for the walk
+    TileBlock tb0;
     if (warp == 0) {
-        const double S = tiles_total(ws, n, smem);
+        load_tile_block(tb0, ws, n, 0, smem);
+        const double S = n <= 32 * kDrawQ ? __shfl_sync(0xffffffffu, tb0.incl, 31) : tiles_total(ws, n, smem);
         if (lane == 0) s_S = S;
     }
     __syncthreads();
@@ -476,13 +483,15 @@ __device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& 
         p_only = true;
         tile_sums_strided<ESZ>(g, rec, true, tv, tv, ws, warp, kWarps);
         __syncthreads();
+        if (warp == 0) load_tile_block(tb0, ws, n, 0, smem);
     }
     if (warp != 0) return;
     const double S = flag ? tiles_total(ws, n, smem) : s_S;
-    const double target = (double)__ldg(g.u_resample + b) * S;
-    int ts = -1;
-    double base = 0.0, carry = 0.0;
-    for (int s0 = 0; s0 < n && ts < 0; s0 += 32 * kDrawQ) {
+    const double target = (double)__shfl_sync(0xffffffffu, ur, 0) * S;
+    double base = 0.0;
+    int ts = walk_tile_block(tb0, 0, 0.0, target, &base);
+    double carry = __shfl_sync(0xffffffffu, tb0.incl, 31);
+    for (int s0 = 32 * kDrawQ; s0 < n && ts < 0; s0 += 32 * kDrawQ) {
         TileBlock tb;
         load_tile_block(tb, ws, n, s0, smem);
         ts = walk_tile_block(tb, s0, carry, target, &base);
@@ -567,6 +576,7 @@ struct FinishSmem {
     int bad[kMaxRows];
     float gath[2 * SV_MAX_GAMMA];
     int status, n;
+    float ur;  // u_resample of the sequence, for the draw
 };
 
 // Finish sequence b with one CTA: warp w folds rows w, w + 8, ... (lane l reads
@@ -622,17 +632,20 @@ __device__ __noinline__ void finish_cta(const PassArgs& g, int b, const SeqIn& i
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
             if (lane == 0) {
-                const bool bad = (MK == -INFINITY) || !isfinite(S) || !(S > 0.0);
-                fs.bad[r] = bad;
+                fs.bad[r] = (MK == -INFINITY) || !isfinite(S) || !(S > 0.0);
                 fs.mk[r] = MK;
                 fs.sum[r] = S;
-                fs.a2[r] = bad ? (double)NAN : (double)MK + log2(S);
             }
         }
     }
     __syncthreads();
 
     if (warp == 0) {
+        // every row's log2-normaliser at once, one row per lane
+        if (!greedy)
+            for (int r = lane; r < rows_used; r += 32)
+                fs.a2[r] = fs.bad[r] ? (double)NAN : (double)fs.mk[r] + log2(fs.sum[r]);
+        __syncwarp();
         int st = 0;
         const int x_j = (lane < gamma) ? in.tok : -1;
         if (!tval) {
@@ -657,9 +670,9 @@ __device__ __noinline__ void finish_cta(const PassArgs& g, int b, const SeqIn& i
             if (greedy) {
                 acc = (x_j == fs.arg[lane]);
             } else {
-                const double Td = (double)T;
-                const double lp = (double)fs.gath[lane] / Td - fs.a2[lane] * kLn2;
-                const double lq = (double)fs.gath[gamma + lane] / Td - fs.a2[gamma + 1 + lane] * kLn2;
+                const double rT = 1.0 / (double)T;
+                const double lp = (double)fs.gath[lane] * rT - fs.a2[lane] * kLn2;
+                const double lq = (double)fs.gath[gamma + lane] * rT - fs.a2[gamma + 1 + lane] * kLn2;
                 acc = log((double)in.ua) < (lp - lq);
             }
         }
@@ -669,20 +682,22 @@ __device__ __noinline__ void finish_cta(const PassArgs& g, int b, const SeqIn& i
         if (lane == 0) {
             fs.status = st;
             fs.n = n;
+            fs.ur = in.ur;
+        }
+        // lane j < gamma holds draft token j (prefetched); entry gamma is never a draft
+        int32_t* ot = a.out_tokens + (size_t)b * (gamma + 1);
+        for (int j = lane; j <= gamma; j += 32) {
+            int v = -1;
+            if (st == 0) {
+                if (j < n) v = x_j;
+                else if (j == n && greedy) v = fs.arg[n];
+            }
+            ot[j] = v;  // a sampled extra token is written by the draw
         }
     }
     __syncthreads();
 
     const int st = fs.status, n = fs.n;
-    int32_t* ot = a.out_tokens + (size_t)b * (gamma + 1);
-    for (int j = tid; j <= gamma; j += kPassThreads) {
-        int v = -1;
-        if (st == 0) {
-            if (j < n) v = __ldg(a.tokens + (size_t)b * gamma + j);
-            else if (j == n && greedy) v = fs.arg[n];
-        }
-        ot[j] = v;  // a sampled extra token is written by the draw
-    }
     if (a.out_log_norm) {
         double* ln = a.out_log_norm + (size_t)b * R;
         for (int r = tid; r < R; r += kPassThreads)
@@ -748,7 +763,8 @@ __global__ void __launch_bounds__(kPassThreads, 2) sv_draw(const __grid_constant
             else tile_range<ESZ, false, kTileBatch>(g, rec, tv, dv, dst, k0, k1);
         }
         cluster.sync();  // every tile sum of b is visible to rank 0
-        if (rank == 0 && rec.mode != kModeNone) pass2_draw<ESZ>(g, b, rec, tiles_in_smem ? s_tiles : dst, tiles_in_smem);
+        if (rank == 0 && rec.mode != kModeNone)
+            pass2_draw<ESZ>(g, b, rec, tiles_in_smem ? s_tiles : dst, tiles_in_smem, s_fin.ur);
         // rank 0's s_rec and s_tiles are rewritten for the next sequence only
         // after the next iteration's finish, which the other ranks wait for
     }

@@ -19,7 +19,9 @@ def main():
     import torch
     assert binding.kernels_per_call(64, 5, 128256, torch.bfloat16) == 3
     cases = [W.make_workload("c2"), W.make_workload("c3", seqs=range(16)),
-             W.make_random(9, 3, 8192, "bf16", seed=77, T=np.array([0.0, 0.7, 1.0] * 3, np.float32))]
+             W.make_random(9, 3, 8192, "bf16", seed=77, T=np.array([0.0, 0.7, 1.0] * 3, np.float32)),
+             W.make_workload("c5", B=600),
+             W.make_random(33, 4, 200, "bf16", seed=78, T=np.array([0.0, 0.7, 1.0] * 11, np.float32))]
     for w in cases:
         st = parity.compare(parity.run_gpu(w), oracle.verify_workload(w))
         print(w.name, st)

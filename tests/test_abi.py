@@ -58,6 +58,7 @@ def test_workspace_size_host_only(lib):
     # otherwise (ticket reset, row pass, resample), 0 on a bad shape
     assert lib.spec_verify_kernels_per_call(64, 5, 128256, 1) == 2
     assert lib.spec_verify_kernels_per_call(3, 2, 3001, 1) == 3
+    assert lib.spec_verify_kernels_per_call(16384, 4, 64, 0) == 1
     assert lib.spec_verify_kernels_per_call(0, 2, 100, 0) == 0
     # a larger batch never needs less workspace
     sizes = [lib.spec_verify_workspace_size(b, 5, 128256, 1) for b in (1, 2, 64, 65, 256)]

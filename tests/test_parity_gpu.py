@@ -43,6 +43,9 @@ RAGGED = [
     (1, 1, 1, "f32"), (3, 2, 7, "bf16"), (5, 3, 9, "f32"), (2, 7, 1000, "bf16"), (4, 1, 1025, "f32"),
     (3, 4, 4097, "bf16"), (17, 5, 3001, "bf16"), (2, 32, 333, "f32"), (6, 3, 33333, "bf16"),
     (1, 4, 32003, "f32"), (9, 2, 8195, "f32"), (40, 2, 257, "bf16"),
+    # rows of at most 256 elements: the short-row kernel with groups of 8, 16 and 32
+    # lanes, mixed greedy / sampled groups in one warp, a part-filled last warp
+    (37, 4, 64, "f32"), (6, 12, 100, "bf16"), (4, 20, 256, "f32"), (11, 8, 33, "bf16"),
 ]
 
 # 16-byte-aligned rows of at least 4 KB: the streaming kernels.  Short rows (one
@@ -77,11 +80,12 @@ def test_aligned_shapes(B, gamma, V, dt):
     parity.assert_parity(st)
 
 
-@pytest.mark.parametrize("V", [300, 4096])
+@pytest.mark.parametrize("V", [64, 300, 4096])
 def test_edge_cases(V):
     """NaN / +inf / all -inf rows, out-of-range tokens, invalid temperatures, masked vocab,
     uniforms outside [0, 1), and residuals that vanish after a rejection
-    (V = 300: the general kernels; V = 4096 f32, 16 KB rows: the streaming kernels)."""
+    (V = 64: the short-row kernel; V = 300: the general kernels; V = 4096 f32, 16 KB
+    rows: the streaming kernels)."""
     import oracle_pins
     rng = np.random.default_rng(9)
     vanished = oracle_pins.vanished_residual_cases(V)
