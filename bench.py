@@ -294,7 +294,7 @@ def run_ours(args):
     w = W.make_workload(WORKLOAD)
     c = Caller(w, dev, lib, binding)
     B, gamma, V, esz = c.B, c.gamma, c.V, c.esz
-    kernel_name = {1: "sv_small (one call: one warp per sequence)",
+    kernel_name = {1: "sv_small (one call: groups of 8, 16 or 32 lanes per sequence)",
                    2: "sv_stream + sv_draw (one call; sv_stream reads every logit once)",
                    3: "sv_reset + sv_rowpass + sv_resample (one call)"}[c.kernels_per_call]
 

@@ -100,7 +100,7 @@ typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
 size_t spec_verify_workspace_size(int B, int gamma, int V, sv_dtype dt);
 
 /* Number of kernel launches one spec_verify() call of this shape enqueues: 1
- * for rows of at most 256 elements (one warp per sequence), 2 for 16-byte-aligned
+ * for rows of at most 256 elements (8, 16 or 32 lanes per sequence), 2 for 16-byte-aligned
  * rows of at least 4 KB (the streaming pass, then the draw), 3 otherwise (ticket
  * reset, row pass, resample); 0 on a bad shape.  Infrastructure: no passage of
  * the pages stands behind it. */

@@ -7,12 +7,13 @@
 //     sequence, sums its draw rows (mostly from L2) and draws.  Used when every
 //     row is 16-byte aligned (V * element size a multiple of 16) and at least
 //     4 KB long.  Every slot these kernels read, the same call wrote.
-//   * sv_small (sv_small.cuh): rows of at most kSmallMaxV elements; one warp per
-//     sequence with the rows in registers, one launch, no workspace traffic.
+//   * sv_small (sv_small.cuh): rows of at most kSmallMaxV elements; a group of
+//     8, 16 or 32 lanes per sequence with the rows in registers, one launch, no
+//     workspace traffic.
 //   * sv_reset + sv_rowpass + sv_resample (sv_generic.cuh): any other shape;
 //     sv_reset zeroes the per-sequence tickets first, so a workspace carries
 //     nothing from one call to the next.
-// SPEC_VERIFY_FORCE_GENERIC=1 in the environment selects the second family for
+// SPEC_VERIFY_FORCE_GENERIC=1 in the environment selects the generic family for
 // every shape (both compute the same results; tests use it to cover both).
 #include "spec_verify.h"
 
