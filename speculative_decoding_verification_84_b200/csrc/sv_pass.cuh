@@ -16,20 +16,23 @@
 //              and are still in L2 when sv_draw reads them; rows streamed earlier
 //              are loaded with an L2 evict-first hint so they do not push them out.
 //   sv_draw    one thread-block cluster per sequence b (clusters loop over the
-//              sequences): rank 0 finishes b -- fp64 combine of the partials
-//              (every load of the finish in flight at once), the log-space
-//              accept test [FlashSpec, Metodologia 1] with the first rejection
-//              from one ballot -- and a cluster barrier hands the outcome to the
-//              cluster through distributed shared memory; the cluster's CTAs then
-//              split the draw rows (residual max(0, p_n - q_n), or p_gamma for
-//              the bonus token) [Speculative Speculative Decoding, Metodologia 2,
-//              "Conceito Central"; Desafios 2, "Amostragem Saguaro"] into tiles
-//              of 32 vectors, one fp32 weight sum per tile into rank 0's shared
-//              memory; after a second barrier rank 0 draws the token by inverse
-//              CDF over the tile sums.
+//              sequences).  Every CTA of the cluster finishes b on its own --
+//              fp64 combine of the partials (every load of the finish in
+//              flight at once), the log-space accept test [FlashSpec,
+//              Metodologia 1] with the first rejection from one ballot -- so no
+//              CTA waits for another to learn the outcome.  The CTAs then split
+//              the draw rows (residual max(0, p_n - q_n), or p_gamma for the bonus
+//              token) [Speculative Speculative Decoding, Metodologia 2, "Conceito
+//              Central"; Desafios 2, "Amostragem Saguaro"] into tiles of 32
+//              vectors, one fp32 weight sum per tile in the CTA's own shared
+//              memory, and send their totals to every CTA through distributed
+//              shared memory.  After one cluster barrier each CTA knows S and
+//              which CTA's range holds u * S; that CTA draws the token by inverse
+//              CDF over its own tile sums, then inside the tile.
 // sv_stream triggers its dependents at entry, so sv_draw's CTAs start as
-// sv_stream's leave; they fetch their sequence's inputs and then wait
-// (griddepcontrol.wait) for all of sv_stream before reading its partials.
+// sv_stream's leave; they fetch their sequence's inputs, take the logarithms and
+// reciprocals those alone decide, and then wait (griddepcontrol.wait) for all of
+// sv_stream before reading its partials.
 // Nothing is carried between calls: every slot a call reads, it wrote.
 #pragma once
 
@@ -47,9 +50,9 @@ constexpr int kStreamVec = 4;                      // 16-byte vectors per lane p
 constexpr int kStreamSlots = 32;                   // partial slots per row (spans >= nq / 31 vectors)
 constexpr int kStreamSpanMin = 128;                // shortest span of a warp (vectors)
 constexpr int kMaxCluster = 8;                     // sv_draw cluster size limit (portable)
-constexpr int kTileSmem = 4096;                    // tile sums kept in rank 0's shared memory up to this many
+constexpr int kTileSmem = 4096;                    // a CTA keeps up to this many tile sums in shared memory
 constexpr int kTileVecs = 32;                      // vectors per tile (one per lane)
-constexpr int kTileBatch = 8;                      // tiles per warp in flight in sv_draw
+constexpr int kTileU = 4;                          // tiles per warp per batch in sv_draw (the next one prefetched)
 constexpr int kStreamMinRowBytes = 4096;           // shorter rows take the generic path
 constexpr int kDrawQ = 16;                         // tile sums per lane per draw block
 
@@ -396,8 +399,8 @@ __device__ long long search_tile(const PassArgs& g, const SeqRec& rec, bool p_on
     double ls = 0.0;
     if (q < g.nq) {
         float xt[VEC], xd[VEC];
-        unpack<ESZ>(ld_stream(tv + q), xt);
-        unpack<ESZ>(p_only ? make_uint4(0u, 0u, 0u, 0u) : ld_stream(dv + q), xd);
+        unpack<ESZ>(__ldg(tv + q), xt);
+        unpack<ESZ>(p_only ? make_uint4(0u, 0u, 0u, 0u) : __ldg(dv + q), xd);
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
             w[e] = weight_of(rec, p_only, xt[e], p_only ? 0.f : xd[e]);
@@ -429,100 +432,37 @@ __device__ long long search_tile(const PassArgs& g, const SeqRec& rec, bool p_on
     return -1;
 }
 
-// Weight sums of tiles k = first, first + stride, ... (< NT2) of the row pair,
-// one warp per tile: lane l takes vector 32k + l; vectors past the row read as
-// -inf target logits, whose weight is 0.
-template <int ESZ>
-__device__ void tile_sums_strided(const PassArgs& g, const SeqRec& rec, bool p_only, const uint4* tv,
-                                  const uint4* dv, float* dst, int first, int stride)
-{
-    constexpr int VEC = 16 / ESZ;
-    const int lane = threadIdx.x & 31;
-    for (int k = first; k < g.NT2; k += stride) {
-        const long long q = (long long)k * kTileVecs + lane;
-        const bool ok = q < g.nq;
-        float xt[VEC], xd[VEC];
-        float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        unpack<ESZ>(ok ? ld_stream(tv + q) : neg_inf_vec<ESZ>(), xt);
-        unpack<ESZ>((ok && !p_only) ? ld_stream(dv + q) : make_uint4(0u, 0u, 0u, 0u), xd);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) w[e] = weight_of(rec, p_only, xt[e], p_only ? 0.f : xd[e]);
-        float s = tree8(w);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) dst[k] = s;
-    }
-}
-
-// Inverse CDF for sequence b, run by the whole CTA (warp 0 does the search): the
-// smallest token k with C_k > u * S over b's tile sums; a vanished residual
-// (S = 0) falls back to p_n, whose tile sums the CTA computes first.
-template <int ESZ>
-__device__ __noinline__ void pass2_draw(const PassArgs& g, int b, const SeqRec& rec, float* ws, bool smem, float ur)
-{
-    __shared__ double s_S;
-    const TailArgs& t = g.t;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = g.NT2;
-    const bool bonus = (rec.mode == kModeBonus);
-    const uint4* tv = reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, rec.n));
-    const uint4* dv = bonus ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
-    // warp 0 keeps the first block of tile sums in registers for the walk
-    TileBlock tb0;
-    if (warp == 0) {
-        load_tile_block(tb0, ws, n, 0, smem);
-        const double S = n <= 32 * kDrawQ ? __shfl_sync(0xffffffffu, tb0.incl, 31) : tiles_total(ws, n, smem);
-        if (lane == 0) s_S = S;
-    }
-    __syncthreads();
-    bool p_only = bonus;
-    int flag = 0;
-    if (!(s_S >= kResidualMin) && !bonus) {
-        // the residual vanished (below kResidualMin): draw from p_n instead
-        flag = SV_ROW_RESIDUAL_ZERO;
-        p_only = true;
-        tile_sums_strided<ESZ>(g, rec, true, tv, tv, ws, warp, kWarps);
-        __syncthreads();
-        if (warp == 0) load_tile_block(tb0, ws, n, 0, smem);
-    }
-    if (warp != 0) return;
-    const double S = flag ? tiles_total(ws, n, smem) : s_S;
-    const double target = (double)__shfl_sync(0xffffffffu, ur, 0) * S;
-    double base = 0.0;
-    int ts = walk_tile_block(tb0, 0, 0.0, target, &base);
-    double carry = __shfl_sync(0xffffffffu, tb0.incl, 31);
-    for (int s0 = 32 * kDrawQ; s0 < n && ts < 0; s0 += 32 * kDrawQ) {
-        TileBlock tb;
-        load_tile_block(tb, ws, n, s0, smem);
-        ts = walk_tile_block(tb, s0, carry, target, &base);
-        carry += __shfl_sync(0xffffffffu, tb.incl, 31);
-    }
-    const long long token = ts >= 0 ? search_tile<ESZ>(g, rec, p_only, tv, dv, ts, base, target) : -1;
-    if (lane == 0) {
-        t.out_tokens[(size_t)b * (t.gamma + 1) + rec.n] = (int)token;
-        if (flag && t.out_status) t.out_status[b] |= flag;
-    }
-}
-
-// Weight sums of tiles [k0, k1) of the row pair, one per warp-tile: warp w takes
-// tiles k0 + 8*(U*j + u) + w (u < U), lane l vector 32k + l, so each lane has U
-// (or 2U, with the draft row) loads in flight.  Vectors past the row read as
-// -inf target logits, whose weight is 0.
+// Weight sums of tiles [k0, k1) of the row pair into dst[k - k0], one per
+// warp-tile: warp w takes tiles k0 + w, k0 + w + 8, ...; lane l vector 32k + l,
+// U tiles per batch.  While a batch is summed the next one is prefetched into
+// L1, so its loads find it there; loads allocate in L1, so the draw's second
+// look at its tile often hits too.  Vectors past the row read as -inf target
+// logits (weight 0).
 template <int ESZ, bool PONLY, int U>
-__device__ void tile_range(const PassArgs& g, const SeqRec& rec, const uint4* tv, const uint4* dv, float* dst,
-                           int k0, int k1)
+__device__ __forceinline__ void tile_sums(const PassArgs& g, const SeqRec& rec, const uint4* tv, const uint4* dv,
+                                          float* dst, int k0, int k1)
 {
     constexpr int VEC = 16 / ESZ;
+    constexpr int STEP = U * kWarps;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int kb = k0 + warp; kb < k1; kb += U * kWarps) {
+    for (int kb = k0 + warp; kb < k1; kb += STEP) {
         uint4 vt[U], vd[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int k = kb + u * kWarps;
             const long long q = (long long)k * kTileVecs + lane;
             const bool ok = k < k1 && q < g.nq;
-            vt[u] = ok ? ld_stream(tv + q) : neg_inf_vec<ESZ>();
-            if (!PONLY) vd[u] = ok ? ld_stream(dv + q) : make_uint4(0u, 0u, 0u, 0u);
+            vt[u] = ok ? __ldg(tv + q) : neg_inf_vec<ESZ>();
+            if (!PONLY) vd[u] = ok ? __ldg(dv + q) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = kb + STEP + u * kWarps;
+            const long long q = (long long)k * kTileVecs + lane;
+            if (k < k1 && q < g.nq) {
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(tv + q));
+                if (!PONLY) asm volatile("prefetch.global.L1 [%0];" ::"l"(dv + q));
+            }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -532,42 +472,74 @@ __device__ void tile_range(const PassArgs& g, const SeqRec& rec, const uint4* tv
             if (!PONLY) unpack<ESZ>(vd[u], xd);
 #pragma unroll
             for (int e = 0; e < VEC; ++e) w[e] = weight_of(rec, PONLY, xt[e], PONLY ? 0.f : xd[e]);
-            float sum = tree8(w);
+            float s = tree8(w);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
             const int k = kb + u * kWarps;
-            if (lane == 0 && k < k1) dst[k] = sum;
+            if (lane == 0 && k < k1) dst[k - k0] = s;
         }
     }
 }
 
-
-// What the finish of one sequence needs from the inputs, fetched before
-// sv_draw waits for sv_stream (lane j < gamma of warp 0 holds position j).
-struct SeqIn {
-    float T;
-    int tok;
-    float ua;
-    float ur;
-};
-
-__device__ __forceinline__ SeqIn load_seq_in(const TailArgs& a, int b)
+// The vanished-residual fallback's tile sums of p_n (rare: kept out of line, so
+// the registers the draw keeps live are saved around it instead of squeezing the
+// main tile loop).
+template <int ESZ>
+__device__ __noinline__ void tile_sums_p(const PassArgs& g, const SeqRec rec, const uint4* tv, float* dst, int k0,
+                                         int k1)
 {
-    const int tid = threadIdx.x;
-    SeqIn in;
-    in.T = __ldg(a.temperature + b);
-    in.tok = -1;
-    in.ua = 0.5f;
-    in.ur = 0.5f;
-    if (tid < a.gamma) {
-        in.tok = __ldg(a.tokens + (size_t)b * a.gamma + tid);
-        in.ua = __ldg(a.u_accept + (size_t)b * a.gamma + tid);
-    }
-    if (tid == 0) in.ur = __ldg(a.u_resample + b);
-    return in;
+    tile_sums<ESZ, true, kTileU>(g, rec, tv, tv, dst, k0, k1);
 }
 
-// Per-row results of the finish (shared memory of rank 0).
+// Per-sequence inputs and what follows from them alone, fetched and computed
+// before sv_draw waits for sv_stream.  Lane j < gamma of every warp holds
+// position j.
+struct SeqPre {
+    float T, khi, klo, ur;
+    double rT;  // 1 / T
+    double lu;  // log u_accept[b][j]
+    int tok;    // draft token x_j
+    int st;     // status bits the inputs alone decide
+};
+
+__device__ __forceinline__ SeqPre seq_pre(const TailArgs& a, int b)
+{
+    const int lane = threadIdx.x & 31;
+    SeqPre s;
+    s.T = __ldg(a.temperature + b);
+    s.ur = __ldg(a.u_resample + b);
+    s.tok = -1;
+    float ua = 0.5f;
+    if (lane < a.gamma) {
+        s.tok = __ldg(a.tokens + (size_t)b * a.gamma + lane);
+        ua = __ldg(a.u_accept + (size_t)b * a.gamma + lane);
+    }
+    const bool greedy = (s.T == 0.f);
+    const bool tval = temperature_ok(s.T);
+    s.khi = 0.f;
+    s.klo = 0.f;
+    s.rT = 0.0;
+    if (tval && !greedy) {
+        split_k(s.T, &s.khi, &s.klo);
+        s.rT = 1.0 / (double)s.T;
+    }
+    s.lu = log((double)ua);
+    int st = 0;
+    if (!tval) {
+        st = SV_ROW_BAD_TEMPERATURE;
+    } else {
+        if (__any_sync(0xffffffffu, lane < a.gamma && (s.tok < 0 || s.tok >= a.V))) st |= SV_ROW_BAD_TOKEN;
+        // the uniforms stand for draws of U[0, 1): anything else (NaN included) is
+        // an invalid input; a greedy sequence reads none
+        if (!greedy && __any_sync(0xffffffffu, (lane < a.gamma && !(ua >= 0.f && ua < 1.f)) ||
+                                                   !(s.ur >= 0.f && s.ur < 1.f)))
+            st |= SV_ROW_BAD_UNIFORM;
+    }
+    s.st = st;
+    return s;
+}
+
+// Per-row results of the finish, in each CTA's shared memory.
 struct FinishSmem {
     double a2[kMaxRows];   // log2-normaliser of each row (NaN if bad)
     double sum[kMaxRows];  // sum relative to the integer offset
@@ -575,26 +547,27 @@ struct FinishSmem {
     int arg[kMaxRows];
     int bad[kMaxRows];
     float gath[2 * SV_MAX_GAMMA];
-    int status, n;
-    float ur;  // u_resample of the sequence, for the draw
+    SeqRec rec;
+    int st;
 };
 
-// Finish sequence b with one CTA: warp w folds rows w, w + 8, ... (lane l reads
-// slot l of each, every load in flight at once) in fp64; gathers log p_j(x_j)
-// and log q_j(x_j) [FlashSpec, Metodologia 1, "Mecanismo"]; warp 0 runs the
-// log-space test at every draft position and takes the first rejection from one
-// ballot; writes the accepted prefix, -1 padding, n_accepted, status and
-// normalisers, and the draw record into *rec_out.
+// Finish sequence b in one CTA (every CTA of the cluster does it, so none waits
+// for another): warp w folds rows w, w + 8, ... (lane l reads slot l of each,
+// every load in flight at once) in fp64; warp 0 forms every row's
+// log2-normaliser (one row per lane), runs the log-space test at every draft
+// position [FlashSpec, Metodologia 1, "Mecanismo"] with the gathered logits, and
+// takes the first rejection from one ballot.  fs.rec and fs.st hold the outcome
+// afterwards.  With `out`, also writes the accepted prefix, -1 padding,
+// n_accepted and the normalisers (the status waits for the draw).
 template <int ESZ>
-__device__ __noinline__ void finish_cta(const PassArgs& g, int b, const SeqIn& in, FinishSmem& fs, SeqRec* rec_out)
+__device__ __forceinline__ void finish_seq(const PassArgs& g, int b, const SeqPre& in, FinishSmem& fs, bool out)
 {
     constexpr int kRowIter = (kMaxRows + kWarps - 1) / kWarps;
     const TailArgs& a = g.t;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gamma = a.gamma, R = a.R;
-    const float T = in.T;
-    const bool greedy = (T == 0.f);
-    const bool tval = temperature_ok(T);
+    const bool greedy = (in.T == 0.f);
+    const bool tval = temperature_ok(in.T);
     const int rows_used = !tval ? 0 : (greedy ? gamma + 1 : R);
 
     const float4* pp = reinterpret_cast<const float4*>(g.part) + (size_t)b * R * kStreamSlots;
@@ -632,141 +605,212 @@ __device__ __noinline__ void finish_cta(const PassArgs& g, int b, const SeqIn& i
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
             if (lane == 0) {
-                fs.bad[r] = (MK == -INFINITY) || !isfinite(S) || !(S > 0.0);
+                const bool bad = (MK == -INFINITY) || !isfinite(S) || !(S > 0.0);
+                fs.bad[r] = bad;
                 fs.mk[r] = MK;
                 fs.sum[r] = S;
+                fs.a2[r] = bad ? (double)NAN : (double)MK + log2(S);
             }
         }
     }
     __syncthreads();
 
     if (warp == 0) {
-        // every row's log2-normaliser at once, one row per lane
-        if (!greedy)
-            for (int r = lane; r < rows_used; r += 32)
-                fs.a2[r] = fs.bad[r] ? (double)NAN : (double)fs.mk[r] + log2(fs.sum[r]);
-        __syncwarp();
-        int st = 0;
-        const int x_j = (lane < gamma) ? in.tok : -1;
-        if (!tval) {
-            st = SV_ROW_BAD_TEMPERATURE;
-        } else {
-            const int badtok = (lane < gamma) && (x_j < 0 || x_j >= a.V);
+        int st = in.st;
+        if (tval) {
             int badrow = 0;
             for (int r = lane; r < rows_used; r += 32) badrow |= fs.bad[r];
-            // the uniforms stand for draws of U[0, 1): anything else (NaN included)
-            // is an invalid input (a greedy sequence reads none)
-            int bad_u = 0;
-            if (!greedy) {
-                if (lane < gamma) bad_u = !(in.ua >= 0.f && in.ua < 1.f);
-                if (lane == 0) bad_u |= !(in.ur >= 0.f && in.ur < 1.f);
-            }
-            if (__any_sync(0xffffffffu, badtok)) st |= SV_ROW_BAD_TOKEN;
             if (__any_sync(0xffffffffu, badrow)) st |= SV_ROW_BAD_LOGITS;
-            if (__any_sync(0xffffffffu, bad_u)) st |= SV_ROW_BAD_UNIFORM;
         }
         bool acc = false;
         if (st == 0 && lane < gamma) {
             if (greedy) {
-                acc = (x_j == fs.arg[lane]);
+                acc = (in.tok == fs.arg[lane]);
             } else {
-                const double rT = 1.0 / (double)T;
-                const double lp = (double)fs.gath[lane] * rT - fs.a2[lane] * kLn2;
-                const double lq = (double)fs.gath[gamma + lane] * rT - fs.a2[gamma + 1 + lane] * kLn2;
-                acc = log((double)in.ua) < (lp - lq);
+                const double lp = (double)fs.gath[lane] * in.rT - fs.a2[lane] * kLn2;
+                const double lq = (double)fs.gath[gamma + lane] * in.rT - fs.a2[gamma + 1 + lane] * kLn2;
+                acc = in.lu < (lp - lq);
             }
         }
         const unsigned mask = (gamma == 32) ? 0xffffffffu : ((1u << gamma) - 1u);
         const unsigned rej = __ballot_sync(0xffffffffu, !acc) & mask;
         const int n = (st != 0) ? 0 : (rej ? __ffs(rej) - 1 : gamma);
         if (lane == 0) {
-            fs.status = st;
-            fs.n = n;
-            fs.ur = in.ur;
-        }
-        // lane j < gamma holds draft token j (prefetched); entry gamma is never a draft
-        int32_t* ot = a.out_tokens + (size_t)b * (gamma + 1);
-        for (int j = lane; j <= gamma; j += 32) {
-            int v = -1;
-            if (st == 0) {
-                if (j < n) v = x_j;
-                else if (j == n && greedy) v = fs.arg[n];
+            SeqRec rec;
+            rec.mode = (st != 0 || greedy) ? kModeNone : (n < gamma ? kModeResidual : kModeBonus);
+            rec.n = n;
+            rec.k_hi = in.khi;
+            rec.k_lo = in.klo;
+            rec.mk_t = 0.f;
+            rec.inv_s_t = 0.f;
+            rec.mk_d = 0.f;
+            rec.inv_s_d = 0.f;
+            if (rec.mode != kModeNone) {
+                rec.mk_t = fs.mk[n];
+                rec.inv_s_t = (float)(1.0 / fs.sum[n]);
+                if (rec.mode == kModeResidual) {
+                    rec.mk_d = fs.mk[gamma + 1 + n];
+                    rec.inv_s_d = (float)(1.0 / fs.sum[gamma + 1 + n]);
+                }
             }
-            ot[j] = v;  // a sampled extra token is written by the draw
+            fs.rec = rec;
+            fs.st = st;
+        }
+        if (out) {
+            // lane j < gamma holds draft token j; entry gamma is never a draft
+            int32_t* ot = a.out_tokens + (size_t)b * (gamma + 1);
+            for (int j = lane; j <= gamma; j += 32) {
+                int v = -1;
+                if (st == 0) {
+                    if (j < n) v = in.tok;
+                    else if (j == n && greedy) v = fs.arg[n];
+                }
+                ot[j] = v;  // a sampled extra token is written by the draw
+            }
+            if (lane == 0) a.out_n[b] = n;
         }
     }
     __syncthreads();
-
-    const int st = fs.status, n = fs.n;
-    if (a.out_log_norm) {
+    if (out && a.out_log_norm) {
         double* ln = a.out_log_norm + (size_t)b * R;
         for (int r = tid; r < R; r += kPassThreads)
-            ln[r] = (tval && !greedy && !fs.bad[r]) ? fs.a2[r] * kLn2 : (double)NAN;
+            ln[r] = (tval && !greedy && r < rows_used && !fs.bad[r]) ? fs.a2[r] * kLn2 : (double)NAN;
     }
-    if (tid == 0) {
-        a.out_n[b] = n;
-        if (a.out_status) a.out_status[b] = st;
-        SeqRec rec;
-        rec.mode = (st != 0 || greedy) ? kModeNone : (n < gamma ? kModeResidual : kModeBonus);
-        rec.n = n;
-        rec.mk_t = 0.f;
-        rec.inv_s_t = 0.f;
-        rec.mk_d = 0.f;
-        rec.inv_s_d = 0.f;
-        rec.k_hi = 0.f;
-        rec.k_lo = 0.f;
-        if (rec.mode != kModeNone) {
-            split_k(T, &rec.k_hi, &rec.k_lo);
-            rec.mk_t = fs.mk[n];
-            rec.inv_s_t = (float)(1.0 / fs.sum[n]);
-            if (rec.mode == kModeResidual) {
-                rec.mk_d = fs.mk[gamma + 1 + n];
-                rec.inv_s_d = (float)(1.0 / fs.sum[gamma + 1 + n]);
-            }
+}
+
+// This CTA's tile sums in w[0, nt): their total (the order the walk uses); warp 0
+// keeps the first block in tb0.
+__device__ __forceinline__ double cta_tiles_total(TileBlock& tb0, const float* w, int nt, bool smem)
+{
+    load_tile_block(tb0, w, nt, 0, smem);
+    return nt <= 32 * kDrawQ ? __shfl_sync(0xffffffffu, tb0.incl, 31) : tiles_total(w, nt, smem);
+}
+
+// The token of the CTA whose tile range holds u * S: walk its tile sums from
+// `base` (the totals of the ranks before it), then the tile (warp 0 only).
+template <int ESZ>
+__device__ long long draw_in_cta(const PassArgs& g, const SeqRec& rec, bool p_only, const uint4* tv,
+                                 const uint4* dv, const TileBlock& tb0, const float* w, int nt, bool smem, int k0,
+                                 double base, double target)
+{
+    double at = 0.0;
+    int ts = walk_tile_block(tb0, 0, base, target, &at);
+    double carry = base + __shfl_sync(0xffffffffu, tb0.incl, 31);
+    for (int s0 = 32 * kDrawQ; s0 < nt && ts < 0; s0 += 32 * kDrawQ) {
+        TileBlock tb;
+        load_tile_block(tb, w, nt, s0, smem);
+        ts = walk_tile_block(tb, s0, carry, target, &at);
+        carry += __shfl_sync(0xffffffffu, tb.incl, 31);
+    }
+    if (ts < 0) {
+        // rounding put u * S past this CTA's last crossing: its last tile with a
+        // positive sum, and in it the last token with a positive weight
+        const int lane = threadIdx.x & 31;
+        int last = -1;
+        for (int kb = nt - 1; kb >= 0 && last < 0; kb -= 32) {
+            const int k = kb - lane;
+            const float v = k >= 0 ? (smem ? w[k] : __ldcg(w + k)) : 0.f;
+            const unsigned m = __ballot_sync(0xffffffffu, v > 0.f);
+            if (m) last = kb - (__ffs(m) - 1);
         }
-        *rec_out = rec;
+        if (last < 0) return -1;
+        return search_tile<ESZ>(g, rec, p_only, tv, dv, k0 + last, 0.0, (double)INFINITY);
     }
+    return search_tile<ESZ>(g, rec, p_only, tv, dv, k0 + ts, at, target);
 }
 
 template <int ESZ>
 __global__ void __launch_bounds__(kPassThreads, 2) sv_draw(const __grid_constant__ PassArgs g)
 {
     __shared__ FinishSmem s_fin;
-    __shared__ SeqRec s_rec;
-    __shared__ float s_tiles[kTileSmem];  // rank 0: b's tile sums, written by the whole cluster
+    __shared__ float s_tiles[kTileSmem];         // this CTA's tile sums
+    __shared__ double s_tot[3][kMaxCluster];     // every rank's total: two alternating, one for the fallback
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank(), cs = (int)cluster.num_blocks();
     const int cid = blockIdx.x / cs, nclusters = gridDim.x / cs;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TailArgs& t = g.t;
-    const bool tiles_in_smem = g.NT2 <= kTileSmem;
-    float* tiles0 = cluster.map_shared_rank(s_tiles, 0);  // rank 0's buffer, from any rank
+    const int per = (g.NT2 + cs - 1) / cs;
+    const int k0 = min(g.NT2, rank * per), k1 = min(g.NT2, k0 + per), nt = k1 - k0;
+    const bool smem = per <= kTileSmem;
 
-    // the first sequence's inputs are not sv_stream's outputs: fetch them before
-    // waiting for sv_stream to complete and its writes to be visible
-    SeqIn in = cid < g.B ? load_seq_in(t, cid) : SeqIn{0.f, -1, 0.5f, 0.5f};
+    // the first sequence's inputs are not sv_stream's outputs: fetch them and work
+    // out what they decide before waiting for sv_stream's writes to be visible
+    SeqPre in = seq_pre(t, min(cid, g.B - 1));
+    cluster.sync();  // every CTA of the cluster runs before any writes another's shared memory
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    for (int b = cid; b < g.B; b += nclusters) {
-        if (b != cid) in = load_seq_in(t, b);
-        if (rank == 0) finish_cta<ESZ>(g, b, in, s_fin, &s_rec);
-        cluster.sync();  // rank 0's outcome is visible to the cluster
-        const SeqRec rec = *cluster.map_shared_rank(&s_rec, 0);
-        float* dst = tiles_in_smem ? tiles0 : g.tsum + (size_t)b * g.NT2;
-        if (rec.mode != kModeNone) {
-            const bool bonus = (rec.mode == kModeBonus);
-            const uint4* tv = reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, rec.n));
-            const uint4* dv = bonus ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
-            // this CTA's share of the tiles
-            const int per = (g.NT2 + cs - 1) / cs;
-            const int k0 = rank * per, k1 = min(g.NT2, k0 + per);
-            if (bonus) tile_range<ESZ, true, kTileBatch>(g, rec, tv, tv, dst, k0, k1);
-            else tile_range<ESZ, false, kTileBatch>(g, rec, tv, dv, dst, k0, k1);
+    int par = 0;
+    for (int b = cid; b < g.B; b += nclusters, par ^= 1) {
+        if (b != cid) {
+            __syncthreads();  // warp 0 is done with the previous sequence's shared memory
+            in = seq_pre(t, b);
         }
-        cluster.sync();  // every tile sum of b is visible to rank 0
-        if (rank == 0 && rec.mode != kModeNone)
-            pass2_draw<ESZ>(g, b, rec, tiles_in_smem ? s_tiles : dst, tiles_in_smem, s_fin.ur);
-        // rank 0's s_rec and s_tiles are rewritten for the next sequence only
-        // after the next iteration's finish, which the other ranks wait for
+        finish_seq<ESZ>(g, b, in, s_fin, rank == 0);
+        const SeqRec rec = s_fin.rec;
+        const bool bonus = (rec.mode == kModeBonus);
+        const uint4* tv = reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, rec.n));
+        const uint4* dv = bonus ? tv : reinterpret_cast<const uint4*>(row_ptr<ESZ>(t, b, t.gamma + 1 + rec.n));
+        float* w = smem ? s_tiles : g.tsum + (size_t)b * g.NT2 + k0;
+        if (rec.mode == kModeResidual) tile_sums<ESZ, false, kTileU>(g, rec, tv, dv, w, k0, k1);
+        else if (rec.mode == kModeBonus) tile_sums<ESZ, true, kTileU>(g, rec, tv, tv, w, k0, k1);
+        __syncthreads();
+        TileBlock tb0;
+        if (warp == 0) {
+            const double tot = rec.mode != kModeNone ? cta_tiles_total(tb0, w, nt, smem) : 0.0;
+            if (lane < cs) *cluster.map_shared_rank(&s_tot[par][rank], lane) = tot;
+        }
+        cluster.sync();  // every rank's total is in every rank's s_tot[par]
+        bool p_only = bonus;
+        int flag = 0;
+        int slot = par;
+        if (rec.mode != kModeNone) {
+            double S = 0.0;
+            for (int r = 0; r < cs; ++r) S += s_tot[slot][r];
+            if (!bonus && !(S >= kResidualMin)) {
+                // the residual vanished (below kResidualMin): draw from p_n instead
+                flag = SV_ROW_RESIDUAL_ZERO;
+                p_only = true;
+                tile_sums_p<ESZ>(g, rec, tv, w, k0, k1);
+                __syncthreads();
+                if (warp == 0) {
+                    const double tot = cta_tiles_total(tb0, w, nt, smem);
+                    if (lane < cs) *cluster.map_shared_rank(&s_tot[2][rank], lane) = tot;
+                }
+                cluster.sync();
+                slot = 2;
+                S = 0.0;
+                for (int r = 0; r < cs; ++r) S += s_tot[slot][r];
+            }
+            // the rank whose range holds u * S (in the sum's own order); if rounding
+            // leaves none, the last rank with a positive total
+            const double target = (double)in.ur * S;
+            double pre = 0.0, base = 0.0;
+            int rs = -1, rl = -1;
+            double basel = 0.0;
+            for (int r = 0; r < cs; ++r) {
+                const double v = s_tot[slot][r];
+                if (rs < 0 && pre + v > target) {
+                    rs = r;
+                    base = pre;
+                }
+                if (v > 0.0) {
+                    rl = r;
+                    basel = pre;
+                }
+                pre += v;
+            }
+            if (rs < 0) {
+                rs = rl;
+                base = basel;
+            }
+            if (rank == rs && warp == 0) {
+                const long long token = draw_in_cta<ESZ>(g, rec, p_only, tv, p_only ? tv : dv, tb0, w, nt, smem, k0,
+                                                         base, target);
+                if (lane == 0) t.out_tokens[(size_t)b * (t.gamma + 1) + rec.n] = (int)token;
+            }
+        }
+        if (rank == 0 && threadIdx.x == 0 && t.out_status) t.out_status[b] = s_fin.st | flag;
     }
 }
 
