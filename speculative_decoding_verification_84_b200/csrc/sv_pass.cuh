@@ -52,7 +52,7 @@ constexpr int kStreamSpanMin = 128;                // shortest span of a warp (v
 constexpr int kMaxCluster = 8;                     // sv_draw cluster size limit (portable)
 constexpr int kTileSmem = 4096;                    // a CTA keeps up to this many tile sums in shared memory
 constexpr int kTileVecs = 32;                      // vectors per tile (one per lane)
-constexpr int kTileU = 4;                          // tiles per warp per batch in sv_draw (the next one prefetched)
+constexpr int kTileU = 4;                          // tiles per warp per batch in sv_draw
 constexpr int kStreamMinRowBytes = 4096;           // shorter rows take the generic path
 constexpr int kDrawQ = 16;                         // tile sums per lane per draw block
 
@@ -434,10 +434,10 @@ __device__ long long search_tile(const PassArgs& g, const SeqRec& rec, bool p_on
 
 // Weight sums of tiles [k0, k1) of the row pair into dst[k - k0], one per
 // warp-tile: warp w takes tiles k0 + w, k0 + w + 8, ...; lane l vector 32k + l,
-// U tiles per batch.  While a batch is summed the next one is prefetched into
-// L1, so its loads find it there; loads allocate in L1, so the draw's second
-// look at its tile often hits too.  Vectors past the row read as -inf target
-// logits (weight 0).
+// U tiles per batch (the CTA's 16 warps per SM keep the loads in flight; an L1
+// prefetch of the next batch measured no faster).  Loads allocate in L1, so the
+// draw's second look at its tile often hits.  Vectors past the row read as -inf
+// target logits (weight 0).
 template <int ESZ, bool PONLY, int U>
 __device__ __forceinline__ void tile_sums(const PassArgs& g, const SeqRec& rec, const uint4* tv, const uint4* dv,
                                           float* dst, int k0, int k1)
@@ -454,15 +454,6 @@ __device__ __forceinline__ void tile_sums(const PassArgs& g, const SeqRec& rec, 
             const bool ok = k < k1 && q < g.nq;
             vt[u] = ok ? __ldg(tv + q) : neg_inf_vec<ESZ>();
             if (!PONLY) vd[u] = ok ? __ldg(dv + q) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int k = kb + STEP + u * kWarps;
-            const long long q = (long long)k * kTileVecs + lane;
-            if (k < k1 && q < g.nq) {
-                asm volatile("prefetch.global.L1 [%0];" ::"l"(tv + q));
-                if (!PONLY) asm volatile("prefetch.global.L1 [%0];" ::"l"(dv + q));
-            }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
