@@ -493,6 +493,21 @@ def c_copies(w):
     return max(3, int(np.ceil(2 * L2_BYTES / w.logits_bytes())) + 1)
 
 
+def run_profile(args):
+    """--profile NAME: warm-up plus K plain calls of workload NAME (c1..c5) and
+    nothing else, so a profiler sees only that workload's launches; no JSON line."""
+    import torch
+    from speculative_decoding_verification_84_b200 import binding, build, workloads as W
+    build.build()
+    lib = binding.load_library()
+    c = Caller(W.make_workload(args.profile), torch.device("cuda", 0), lib, binding)
+    for i in range(args.warmup + args.steps):
+        c.call(i)
+    torch.cuda.synchronize()
+    print(f"{args.profile}: {args.warmup + args.steps} calls, {c.kernels_per_call} launches each", flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -502,7 +517,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="skip the line's per-workload numbers")
+    ap.add_argument("--profile", choices=PER_CONFIG, default=None,
+                    help="only make warm-up + K calls of this workload (for a profiler); no JSON line")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile(args)
     if args.impl == "reference":
         if args.steps > 200:
             args.steps = 20
