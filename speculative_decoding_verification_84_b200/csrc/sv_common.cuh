@@ -379,6 +379,41 @@ __device__ __forceinline__ void amax_merge(Amax& a, float best, int idx, int nan
     a.nan |= nan;
 }
 
+// A 16-byte vector whose first element has index i0, folded into a first argmax
+// that has seen only lower indices: the vector's maximum (NaN ignored), and only
+// when it beats a.best the first element equal to it; a NaN anywhere makes the
+// sum of the elements NaN (so does +inf with -inf, in a row the +inf already
+// makes bad).  A few instructions per vector instead of a few per element.
+template <int ESZ>
+__device__ __forceinline__ void amax_vec(Amax& a, const uint4& v, int i0)
+{
+    constexpr int VEC = 16 / ESZ;
+    const float m = vec_max<ESZ>(v);
+    if (ESZ == 2) {
+        const __nv_bfloat162 s0 = __hadd2(*reinterpret_cast<const __nv_bfloat162*>(&v.x),
+                                          *reinterpret_cast<const __nv_bfloat162*>(&v.y));
+        const __nv_bfloat162 s1 = __hadd2(*reinterpret_cast<const __nv_bfloat162*>(&v.z),
+                                          *reinterpret_cast<const __nv_bfloat162*>(&v.w));
+        const __nv_bfloat162 s2 = __hadd2(s0, s1);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(&s2);
+        const float t = bf16_lo(w) + bf16_hi(w);
+        a.nan |= (t != t);
+    } else {
+        const float t = (__uint_as_float(v.x) + __uint_as_float(v.y)) + (__uint_as_float(v.z) + __uint_as_float(v.w));
+        a.nan |= (t != t);
+    }
+    if (m > a.best) {
+        float x[VEC];
+        unpack<ESZ>(v, x);
+        int k = VEC - 1;
+#pragma unroll
+        for (int e = VEC - 1; e >= 0; --e)
+            if (x[e] == m) k = e;
+        a.best = m;
+        a.idx = i0 + k;
+    }
+}
+
 // ---- block reductions over kThreads threads
 __device__ __forceinline__ double warp_sum(double v)
 {

@@ -216,16 +216,10 @@ __device__ __forceinline__ void stream_segment(const PassArgs& g, int b, int r, 
                 const int i = j0 + u * 32 + lane;
                 v[u] = i < n ? ld_stream(p + i) : neg_inf_vec<ESZ>();
             }
+            // a lane meets its vectors in increasing index order; fill vectors
+            // (-inf past the segment) never beat a real maximum
 #pragma unroll
-            for (int u = 0; u < kStreamVec; ++u) {
-                float xv[VEC];
-                unpack<ESZ>(v[u], xv);
-                const int i0 = e0 + (j0 + u * 32 + lane) * VEC;
-                // fill elements (-inf past the segment) have larger indices than
-                // the real ones, so they never win a tie
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) amax_add(A, xv[e], i0 + e);
-            }
+            for (int u = 0; u < kStreamVec; ++u) amax_vec<ESZ>(A, v[u], e0 + (j0 + u * 32 + lane) * VEC);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
