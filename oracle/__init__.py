@@ -49,6 +49,13 @@ def load_library(path: str):
                                      ctypes.c_int]
     lib.sv_oracle_verify.restype = ctypes.c_int
     lib.sv_oracle_max_threads.restype = ctypes.c_int
+    lib.sv_oracle_fanout.argtypes = [ctypes.c_double, ctypes.c_int, ctypes.c_int, p]
+    lib.sv_oracle_fanout.restype = ctypes.c_int
+    lib.sv_oracle_topf.argtypes = [p, p, ctypes.c_int, p, ctypes.c_int, ctypes.c_int, ctypes.c_int, p, p, p,
+                                   ctypes.c_int]
+    lib.sv_oracle_topf.restype = ctypes.c_int
+    lib.sv_oracle_cache_lookup.argtypes = [p, p, p, ctypes.c_int, ctypes.c_int, p, p]
+    lib.sv_oracle_cache_lookup.restype = ctypes.c_int
     return lib
 
 
@@ -119,3 +126,55 @@ def verify_workload(w, n_threads: int = 0) -> OracleResult:
     """Run the oracle on a ``Workload`` from the seeded generators."""
     return verify(w.target, w.draft, w.draft_tokens, w.temperature, w.u_accept, w.u_resample,
                   bf16=(w.dtype == "bf16"), n_threads=n_threads)
+
+
+def fanout(alpha: float, gamma: int, budget: int, lib=None) -> np.ndarray:
+    """Cache slots F_n per outcome n in [0, gamma]: geometric in n with acceptance
+    rate alpha, summing to the budget (see ``sv_oracle.c``)."""
+    lib = _load() if lib is None else lib
+    F = np.empty((gamma + 1,), dtype=np.int32)
+    if lib.sv_oracle_fanout(float(alpha), int(gamma), int(budget), _ptr(F)) != 0:
+        raise ValueError("bad fan-out arguments")
+    return F
+
+
+def topf(target: np.ndarray, draft: np.ndarray, temperature: np.ndarray, F, *, bf16: bool | None = None,
+         n_threads: int = 0, lib=None):
+    """Top-F_n tokens of the extra token's distribution for every outcome n, and
+    their probabilities: ([B, sum F] int32, [B, sum F] float64)."""
+    lib = _load() if lib is None else lib
+    target = np.ascontiguousarray(target)
+    draft = np.ascontiguousarray(draft)
+    if bf16 is None:
+        bf16 = target.dtype == np.uint16
+    B, g1, V = target.shape
+    gamma = g1 - 1
+    F = np.ascontiguousarray(F, dtype=np.int32).reshape(gamma + 1)
+    T = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    Ft = int(F.sum())
+    tok = np.empty((B, Ft), dtype=np.int32)
+    prob = np.empty((B, Ft), dtype=np.float64)
+    rc = lib.sv_oracle_topf(_ptr(target), _ptr(draft), int(bool(bf16)), _ptr(T), B, gamma, V, _ptr(F),
+                            _ptr(tok), _ptr(prob), int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"sv_oracle_topf failed ({rc})")
+    return tok, prob
+
+
+def topf_workload(w, F, n_threads: int = 0):
+    return topf(w.target, w.draft, w.temperature, F, bf16=(w.dtype == "bf16"), n_threads=n_threads)
+
+
+def cache_lookup(out_tokens: np.ndarray, out_n: np.ndarray, cache: np.ndarray, F, lib=None) -> np.ndarray:
+    """Slot of each sequence's outcome (n, extra token) in its cache, else -1."""
+    lib = _load() if lib is None else lib
+    out_tokens = np.ascontiguousarray(out_tokens, dtype=np.int32)
+    B, g1 = out_tokens.shape
+    gamma = g1 - 1
+    out_n = np.ascontiguousarray(out_n, dtype=np.int32).reshape(B)
+    F = np.ascontiguousarray(F, dtype=np.int32).reshape(gamma + 1)
+    cache = np.ascontiguousarray(cache, dtype=np.int32).reshape(B, int(F.sum()))
+    slot = np.empty((B,), dtype=np.int32)
+    if lib.sv_oracle_cache_lookup(_ptr(out_tokens), _ptr(out_n), _ptr(cache), B, gamma, _ptr(F), _ptr(slot)) != 0:
+        raise RuntimeError("sv_oracle_cache_lookup failed")
+    return slot

@@ -300,3 +300,179 @@ int sv_oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * The speculation cache's side of the outcome [Speculative Speculative Decoding,
+ * Metodologia 2, "Conceito Central" (the verification outcome is the number
+ * accepted plus one more token, and the cache holds speculations for likely
+ * outcomes); Desafios 1 (a geometric fan-out over the accepted lengths within a
+ * budget) and 2 (the extra token after a rejection comes from the residual, and
+ * Saguaro sampling puts residual mass on the cached top-F tokens)].
+ *
+ * sv_oracle_fanout: F_n for n in [0, gamma] from an acceptance rate alpha in
+ * [0, 1] and a budget of cache slots.  P(n) = alpha^n (1 - alpha) for n < gamma and
+ * alpha^gamma for n = gamma -- the law of the accepted length when every position
+ * accepts with probability alpha; F_n = floor(budget * P(n)), then one more slot
+ * to each n in decreasing order of budget * P(n) - F_n (ties: smaller n) until the
+ * F_n add up to the budget.
+ *
+ * sv_oracle_topf: for sequence b and outcome n, the distribution the extra token
+ * is drawn from after that outcome -- norm(max(0, p_n - q_n)) for n < gamma (p_n
+ * when the residual mass is below 2^-18, as the draw does), p_gamma for n =
+ * gamma; with T == 0 a point mass on the first argmax of target row n -- and its
+ * F_n most probable tokens in decreasing probability (equal probabilities:
+ * smaller token first), with their probabilities.  Slots past the tokens of
+ * positive probability hold -1 and 0.  Sequences with an invalid temperature or
+ * a bad row (status 4 or 2 as in sv_oracle_verify) hold -1 and 0 everywhere.
+ * Outcome n's slots are [off_n, off_n + F_n), off_n = F_0 + ... + F_{n-1}.
+ *
+ * sv_oracle_cache_lookup: for sequence b with outcome n = out_n[b] and extra
+ * token out_tokens[b][n], the slot s in [off_n, off_n + F_n) with
+ * cache[b][s] == that token (the first one), else -1; -1 too when the sequence
+ * emitted no extra token (-1).
+ */
+int sv_oracle_fanout(double alpha, int gamma, int budget, int32_t* F)
+{
+    if (gamma < 1 || gamma > 32 || budget < 0 || !(alpha >= 0.0 && alpha <= 1.0)) return -1;
+    double want[33];
+    int total = 0;
+    for (int n = 0; n <= gamma; ++n) {
+        const double P = n < gamma ? pow(alpha, n) * (1.0 - alpha) : pow(alpha, gamma);
+        want[n] = (double)budget * P;
+        F[n] = (int32_t)floor(want[n]);
+        total += F[n];
+    }
+    while (total < budget) { /* largest remainder first, smaller n on ties */
+        int best = 0;
+        double br = -1.0;
+        for (int n = 0; n <= gamma; ++n) {
+            const double rem = want[n] - (double)F[n];
+            if (rem > br) { br = rem; best = n; }
+        }
+        F[best] += 1;
+        want[best] -= 1.0; /* its remainder is used up */
+        total += 1;
+    }
+    return 0;
+}
+
+typedef struct { double w; int v; } WTok;
+
+static int wtok_cmp(const void* a, const void* b)
+{
+    const WTok* x = (const WTok*)a;
+    const WTok* y = (const WTok*)b;
+    if (x->w > y->w) return -1;
+    if (x->w < y->w) return 1;
+    return (x->v > y->v) - (x->v < y->v);
+}
+
+static void topf_one(const void* tgt, const void* dft, int is_bf16, double T, int gamma, int V, size_t b,
+                     const int32_t* F, int Ftot, int32_t* out_tok, double* out_p, WTok* buf)
+{
+    for (int s = 0; s < Ftot; ++s) { out_tok[s] = -1; out_p[s] = 0.0; }
+    if (!(T == 0.0 || (isfinite(T) && T >= ORACLE_T_MIN))) return;
+    const size_t trow0 = b * (size_t)(gamma + 1) * (size_t)V;
+    const size_t drow0 = b * (size_t)gamma * (size_t)V;
+    if (T == 0.0) {
+        int arg[33];
+        for (int j = 0; j <= gamma; ++j) {
+            arg[j] = row_argmax(tgt, is_bf16, trow0 + (size_t)j * V, V);
+            if (arg[j] < 0) return;
+        }
+        int off = 0;
+        for (int n = 0; n <= gamma; ++n) {
+            if (F[n] > 0) { out_tok[off] = arg[n]; out_p[off] = 1.0; }
+            off += F[n];
+        }
+        return;
+    }
+    double lse_t[33], lse_d[32];
+    for (int j = 0; j <= gamma; ++j)
+        if (!row_lse(tgt, is_bf16, trow0 + (size_t)j * V, V, T, &lse_t[j])) return;
+    for (int j = 0; j < gamma; ++j)
+        if (!row_lse(dft, is_bf16, drow0 + (size_t)j * V, V, T, &lse_d[j])) return;
+    int off = 0;
+    for (int n = 0; n <= gamma; ++n) {
+        double S = 0.0;
+        for (int v = 0; v < V; ++v) {
+            const double pt = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);
+            const double qd = n < gamma ? exp(widen(dft, is_bf16, drow0 + (size_t)n * V + v) / T - lse_d[n]) : 0.0;
+            buf[v].w = n < gamma ? fmax(0.0, pt - qd) : pt;
+            buf[v].v = v;
+            S += buf[v].w;
+        }
+        if (n < gamma && !(ORACLE_RESIDUAL_MIN <= S)) { /* the residual vanished: p_n, as the draw */
+            S = 0.0;
+            for (int v = 0; v < V; ++v) {
+                buf[v].w = exp(widen(tgt, is_bf16, trow0 + (size_t)n * V + v) / T - lse_t[n]);
+                S += buf[v].w;
+            }
+        }
+        qsort(buf, (size_t)V, sizeof(WTok), wtok_cmp);
+        for (int s = 0; s < F[n] && s < V; ++s) {
+            if (!(buf[s].w > 0.0)) break;
+            out_tok[off + s] = buf[s].v;
+            out_p[off + s] = buf[s].w / S;
+        }
+        off += F[n];
+    }
+}
+
+/*
+ * target: [B][gamma+1][V], draft: [B][gamma][V] (is_bf16 selects uint16 bf16 bits);
+ * F: [gamma+1] slots per outcome.  Outputs: out_tokens [B][sum F] int32 and out_prob
+ * [B][sum F] double.  Returns 0, or -1 on a bad shape.
+ */
+int sv_oracle_topf(const void* target, const void* draft, int is_bf16, const float* temperature, int B,
+                   int gamma, int V, const int32_t* F, int32_t* out_tokens, double* out_prob, int n_threads)
+{
+    if (B < 0 || gamma < 1 || gamma > 32 || V < 1) return -1;
+    int Ftot = 0;
+    for (int n = 0; n <= gamma; ++n) {
+        if (F[n] < 0) return -1;
+        Ftot += F[n];
+    }
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        WTok* buf = (WTok*)malloc(sizeof(WTok) * (size_t)V);
+        if (!buf) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b) {
+            if (!buf) continue;
+            topf_one(target, draft, is_bf16, (double)temperature[b], gamma, V, (size_t)b, F, Ftot,
+                     out_tokens + (size_t)b * Ftot, out_prob + (size_t)b * Ftot, buf);
+        }
+        free(buf);
+    }
+    return failed ? -2 : 0;
+}
+
+int sv_oracle_cache_lookup(const int32_t* out_tokens, const int32_t* out_n, const int32_t* cache, int B,
+                           int gamma, const int32_t* F, int32_t* out_slot)
+{
+    if (B < 0 || gamma < 1 || gamma > 32) return -1;
+    int off[34];
+    off[0] = 0;
+    for (int n = 0; n <= gamma; ++n) off[n + 1] = off[n] + F[n];
+    const int Ftot = off[gamma + 1];
+    for (int b = 0; b < B; ++b) {
+        out_slot[b] = -1;
+        const int n = out_n[b];
+        if (n < 0 || n > gamma) continue;
+        const int x = out_tokens[(size_t)b * (gamma + 1) + n];
+        if (x < 0) continue;
+        for (int s = off[n]; s < off[n + 1]; ++s)
+            if (cache[(size_t)b * Ftot + s] == x) { out_slot[b] = s; break; }
+    }
+    return 0;
+}

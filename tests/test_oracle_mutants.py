@@ -48,10 +48,25 @@ MUTANTS = {
         "double lp = widen(tgt, is_bf16, trow0 + (size_t)j * V + (size_t)tok[j]) / T - lse_d[j];"),
 }
 
+# planted mistakes in the speculation-cache functions, caught by topf_pins
+TOPF_MUTANTS = {
+    "topf_ascending": ("if (x->w > y->w) return -1;\n    if (x->w < y->w) return 1;",
+                       "if (x->w > y->w) return 1;\n    if (x->w < y->w) return -1;"),
+    "topf_ties_larger_token_first": ("return (x->v > y->v) - (x->v < y->v);", "return (x->v < y->v) - (x->v > y->v);"),
+    "topf_residual_not_clamped": ("buf[v].w = n < gamma ? fmax(0.0, pt - qd) : pt;", "buf[v].w = n < gamma ? pt - qd : pt;"),
+    "topf_no_vanished_fallback": ("if (n < gamma && !(ORACLE_RESIDUAL_MIN <= S)) {", "if (0) {"),
+    "topf_unnormalised": ("out_p[off + s] = buf[s].w / S;", "out_p[off + s] = buf[s].w;"),
+    "topf_keeps_zero_weights": ("if (!(buf[s].w > 0.0)) break;", ";"),
+    "fanout_uniform": ("const double P = n < gamma ? pow(alpha, n) * (1.0 - alpha) : pow(alpha, gamma);",
+                       "const double P = 1.0 / (double)(gamma + 1);"),
+    "fanout_remainder_to_last": ("if (rem > br) { br = rem; best = n; }", "if (rem >= br) { br = rem; best = n; }"),
+    "lookup_wrong_outcome_slots": ("for (int s = off[n]; s < off[n + 1]; ++s)", "for (int s = 0; s < Ftot; ++s)"),
+}
+
 
 def _build_mutant(name, tmpdir):
     src = open(SRC).read()
-    old, new = MUTANTS[name]
+    old, new = {**MUTANTS, **TOPF_MUTANTS}[name]
     assert src.count(old) == 1, f"mutation site for {name} not unique"
     path = os.path.join(tmpdir, f"{name}.c")
     with open(path, "w") as f:
@@ -82,4 +97,39 @@ def test_mutant_is_caught(name):
                 P.check_bonus_distribution(verify, min_samples=3000)
             except Exception as e:  # noqa: BLE001
                 caught.append(("check_bonus_distribution", type(e).__name__))
+        assert caught, f"planted mistake {name} passed every pin"
+
+
+class _OracleWith:
+    """The oracle's Python functions bound to a mutant library."""
+
+    def __init__(self, lib):
+        self.lib = lib
+
+    def verify(self, *a, **k):
+        return oracle.verify(*a, lib=self.lib, **k)
+
+    def topf(self, *a, **k):
+        return oracle.topf(*a, lib=self.lib, **k)
+
+    def fanout(self, *a, **k):
+        return oracle.fanout(*a, lib=self.lib, **k)
+
+    def cache_lookup(self, *a, **k):
+        return oracle.cache_lookup(*a, lib=self.lib, **k)
+
+
+@pytest.mark.parametrize("name", sorted(TOPF_MUTANTS))
+def test_topf_mutant_is_caught(name):
+    import topf_pins as TP
+    with tempfile.TemporaryDirectory() as d:
+        O = _OracleWith(_build_mutant(name, d))
+        caught = []
+        for check in TP.ALL_TOPF_CHECKS:
+            try:
+                with np.errstate(all="ignore"):
+                    check(O)
+            except Exception as e:  # noqa: BLE001 - any failure counts as caught
+                caught.append((check.__name__, type(e).__name__))
+                break
         assert caught, f"planted mistake {name} passed every pin"
