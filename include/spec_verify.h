@@ -188,6 +188,71 @@ sv_status spec_verify_noalloc(const void* target_logits, const void* draft_logit
                               double* out_log_norm, int32_t* out_row_status,
                               struct CUstream_st* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * The speculation cache's side of an outcome [Speculative Speculative
+ * Decoding, Metodologia 2, "Conceito Central": a verification outcome is the
+ * number of accepted drafts plus one more token, and the cache holds
+ * speculations for likely outcomes; Desafios 1: a geometric fan-out of cache
+ * slots over the accepted lengths within a budget; Desafios 2: the extra token
+ * after a rejection follows the residual distribution, and the cached tokens
+ * are its most probable ones].
+ */
+
+/* Most cache slots one outcome can have in spec_verify_topf. */
+#define SV_MAX_TOPF 32
+
+/* Cache slots per outcome n in [0, gamma], on the host: outcome n has share
+ * alpha^n (1 - alpha) (n < gamma) or alpha^gamma (n = gamma) of the budget -- the
+ * law of the accepted length when each position accepts with probability alpha
+ * -- rounded down, and the slots left over go one each to the largest
+ * remainders (the smaller n on ties).  fanout: host int32[gamma + 1].
+ * Returns SV_ERR_INVALID_ARG for alpha outside [0, 1], gamma outside
+ * [1, SV_MAX_GAMMA], a negative budget or a null pointer. */
+sv_status spec_verify_fanout(double alpha, int gamma, int budget, int32_t* fanout);
+
+/*
+ * For every sequence b and outcome n with fanout[n] > 0, the fanout[n] most
+ * probable tokens of the distribution spec_verify draws the extra token from
+ * after outcome n: norm(max(0, p_n - q_n)) for n < gamma (p_n when that residual
+ * mass is below 2^-18, as spec_verify does), p_gamma for n = gamma, and for
+ * T = 0 a point mass on the first argmax of target row n; in decreasing
+ * probability, equal probabilities smaller token first, with the probabilities.
+ * Slots past the tokens of positive probability hold -1 and 0; sequences whose
+ * row_status has SV_ROW_BAD_TEMPERATURE or SV_ROW_BAD_LOGITS hold -1 and 0
+ * everywhere.  Outcome n's slots are [off_n, off_n + fanout[n]) of each row,
+ * off_n = fanout[0] + ... + fanout[n-1].
+ *
+ *   target_logits, draft_logits, dt, temperature  as for spec_verify
+ *   log_norm      [B][2*gamma+1] double and row_status [B] int32: spec_verify's
+ *                 out_log_norm and out_row_status for the same inputs (p and q
+ *                 are formed from these normalisers: one pass over the rows)
+ *   fanout        HOST int32[gamma + 1], each in [0, SV_MAX_TOPF]
+ *   out_tokens    [B][sum fanout] int32;  out_prob [B][sum fanout] float
+ *
+ * Device pointers are caller-owned; nothing is allocated, no workspace.
+ * Host-checkable errors return before any launch.  Infrastructure around the
+ * passages above; the selection rule (most probable first, smaller token on
+ * ties) is this library's reading.
+ */
+sv_status spec_verify_topf(const void* target_logits, const void* draft_logits, sv_dtype dt,
+                           const float* temperature, const double* log_norm, const int32_t* row_status,
+                           const int32_t* fanout, int B, int gamma, int V, int32_t* out_tokens,
+                           float* out_prob, struct CUstream_st* stream);
+
+/*
+ * Whether each sequence's outcome is in its cache: out_slot[b] = the first slot
+ * s of outcome n's range (n = out_n_accepted[b]) with cache_tokens[b][s] equal to
+ * the extra token out_tokens[b][n], else -1 (also when that token is -1).
+ *   out_tokens [B][gamma+1], out_n_accepted [B]: spec_verify's outputs;
+ *   cache_tokens [B][sum fanout] (e.g. spec_verify_topf's out_tokens);
+ *   fanout HOST int32[gamma + 1]; out_slot [B] int32.  All device pointers but
+ *   fanout.
+ */
+sv_status spec_verify_cache_lookup(const int32_t* out_tokens, const int32_t* out_n_accepted,
+                                   const int32_t* cache_tokens, const int32_t* fanout, int B, int gamma,
+                                   int32_t* out_slot, struct CUstream_st* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,7 +20,9 @@ SV_OK = 0
 SV_DTYPE_F32, SV_DTYPE_BF16 = 0, 1
 ROW_BAD_TOKEN, ROW_BAD_LOGITS, ROW_BAD_TEMPERATURE, ROW_RESIDUAL_ZERO, ROW_BAD_UNIFORM = 1, 2, 4, 8, 16
 EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_init",
-            "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc")
+            "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc",
+            "spec_verify_fanout", "spec_verify_topf", "spec_verify_cache_lookup")
+MAX_TOPF = 32
 
 _lib = None
 
@@ -52,6 +54,12 @@ def load_library(path: str = LIB_PATH):
     lib.spec_verify_kernels_per_call.restype = i32
     lib.spec_verify_status_string.argtypes = [i32]
     lib.spec_verify_status_string.restype = ctypes.c_char_p
+    lib.spec_verify_fanout.argtypes = [ctypes.c_double, i32, i32, vp]
+    lib.spec_verify_fanout.restype = i32
+    lib.spec_verify_topf.argtypes = [vp, vp, i32, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
+    lib.spec_verify_topf.restype = i32
+    lib.spec_verify_cache_lookup.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp]
+    lib.spec_verify_cache_lookup.restype = i32
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -161,6 +169,72 @@ def verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Tensor
     if return_row_status:
         out.append(row_status)
     return tuple(out)
+
+
+def fanout(alpha: float, gamma: int, budget: int):
+    """Cache slots per outcome n in [0, gamma] (host int32 array): geometric in n
+    with acceptance rate alpha, summing to the budget."""
+    import numpy as np
+    F = np.empty((gamma + 1,), dtype=np.int32)
+    st = load_library().spec_verify_fanout(float(alpha), int(gamma), int(budget), F.ctypes.data)
+    if st != SV_OK:
+        raise SpecVerifyError(st, status_string(st))
+    return F
+
+
+def _host_fanout(F, gamma):
+    import numpy as np
+    F = np.ascontiguousarray(F, dtype=np.int32).reshape(gamma + 1)
+    return F, int(F.sum())
+
+
+def topf(target: torch.Tensor, draft: torch.Tensor, temperature: torch.Tensor, log_norm: torch.Tensor,
+         row_status: torch.Tensor, F, *, stream: torch.cuda.Stream | None = None):
+    """Top-F_n tokens of the extra token's distribution for every outcome n, from
+    spec_verify's log_norm and row_status: (tokens [B, sum F] int32, prob [B, sum F]
+    float32) on the device."""
+    lib = load_library()
+    device = target.device
+    B, g1, V = target.shape
+    gamma = g1 - 1
+    dt = _dt_code(target.dtype)
+    _check(target, "target", None, (B, gamma + 1, V), device)
+    _check(draft, "draft", target.dtype, (B, gamma, V), device)
+    _check(temperature, "temperature", torch.float32, (B,), device)
+    _check(log_norm, "log_norm", torch.float64, (B, 2 * gamma + 1), device)
+    _check(row_status, "row_status", torch.int32, (B,), device)
+    Fh, Ft = _host_fanout(F, gamma)
+    tok = torch.empty((B, Ft), dtype=torch.int32, device=device)
+    prob = torch.empty((B, Ft), dtype=torch.float32, device=device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        st = lib.spec_verify_topf(target.data_ptr(), draft.data_ptr(), dt, temperature.data_ptr(),
+                                  log_norm.data_ptr(), row_status.data_ptr(), Fh.ctypes.data, B, gamma, V,
+                                  tok.data_ptr(), prob.data_ptr(), s.cuda_stream)
+    if st != SV_OK:
+        raise SpecVerifyError(st, status_string(st))
+    return tok, prob
+
+
+def cache_lookup(out_tokens: torch.Tensor, n_accepted: torch.Tensor, cache_tokens: torch.Tensor, F, *,
+                 stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Slot of each sequence's outcome (n, extra token) in its cache, else -1 ([B] int32)."""
+    lib = load_library()
+    device = out_tokens.device
+    B, g1 = out_tokens.shape
+    gamma = g1 - 1
+    Fh, Ft = _host_fanout(F, gamma)
+    _check(out_tokens, "out_tokens", torch.int32, (B, gamma + 1), device)
+    _check(n_accepted, "n_accepted", torch.int32, (B,), device)
+    _check(cache_tokens, "cache_tokens", torch.int32, (B, Ft), device)
+    slot = torch.empty((B,), dtype=torch.int32, device=device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        st = lib.spec_verify_cache_lookup(out_tokens.data_ptr(), n_accepted.data_ptr(), cache_tokens.data_ptr(),
+                                          Fh.ctypes.data, B, gamma, slot.data_ptr(), s.cuda_stream)
+    if st != SV_OK:
+        raise SpecVerifyError(st, status_string(st))
+    return slot
 
 
 def to_device(w, device="cuda"):

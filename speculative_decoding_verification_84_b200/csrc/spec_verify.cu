@@ -29,6 +29,7 @@
 #include "sv_generic.cuh"
 #include "sv_pass.cuh"
 #include "sv_small.cuh"
+#include "sv_topf.cuh"
 
 namespace {
 
@@ -524,4 +525,102 @@ extern "C" sv_status spec_verify_noalloc(const void* target_logits, const void* 
             : launch<4>(p, target_logits, draft_logits, draft_tokens, temperature, u_accept, u_resample, out_tokens,
                         out_n_accepted, out_log_norm, out_row_status, ws, st);
     return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------------- speculation cache
+
+extern "C" sv_status spec_verify_fanout(double alpha, int gamma, int budget, int32_t* fanout)
+{
+    if (!fanout || gamma < 1 || gamma > SV_MAX_GAMMA || budget < 0 || !(alpha >= 0.0 && alpha <= 1.0))
+        return SV_ERR_INVALID_ARG;
+    // share of outcome n: alpha^n (1 - alpha), n < gamma; alpha^gamma for n = gamma
+    double share[SV_MAX_GAMMA + 1];
+    double an = 1.0;
+    int given = 0;
+    for (int n = 0; n <= gamma; ++n) {
+        share[n] = (double)budget * (n < gamma ? an * (1.0 - alpha) : an);
+        an *= alpha;
+        fanout[n] = (int32_t)share[n];  // share >= 0: the cast rounds down
+        given += fanout[n];
+    }
+    // the slots left over go one each to the largest remainders (smaller n first)
+    while (given < budget) {
+        int pick = 0;
+        double most = -1.0;
+        for (int n = 0; n <= gamma; ++n)
+            if (share[n] - (double)fanout[n] > most) {
+                most = share[n] - (double)fanout[n];
+                pick = n;
+            }
+        ++fanout[pick];
+        share[pick] -= 1.0;
+        ++given;
+    }
+    return SV_OK;
+}
+
+namespace {
+
+bool fill_topf_args(const int32_t* fanout, int B, int gamma, int V, sv::TopfArgs* g)
+{
+    if (!fanout || B < 1 || gamma < 1 || gamma > SV_MAX_GAMMA || V < 1 || V > SV_MAX_V) return false;
+    g->B = B;
+    g->gamma = gamma;
+    g->V = V;
+    g->off[0] = 0;
+    g->n_nz = 0;
+    for (int n = 0; n <= gamma; ++n) {
+        if (fanout[n] < 0 || fanout[n] > SV_MAX_TOPF) return false;
+        g->F[n] = fanout[n];
+        g->off[n + 1] = g->off[n] + fanout[n];
+        if (fanout[n] > 0) g->nz[g->n_nz++] = n;
+    }
+    g->Ftot = g->off[gamma + 1];
+    return true;
+}
+
+}  // namespace
+
+extern "C" sv_status spec_verify_topf(const void* target_logits, const void* draft_logits, sv_dtype dt,
+                                      const float* temperature, const double* log_norm, const int32_t* row_status,
+                                      const int32_t* fanout, int B, int gamma, int V, int32_t* out_tokens,
+                                      float* out_prob, struct CUstream_st* stream)
+{
+    if (dt != SV_DTYPE_F32 && dt != SV_DTYPE_BF16) return SV_ERR_UNSUPPORTED_DTYPE;
+    sv::TopfArgs g;
+    if (!fill_topf_args(fanout, B, gamma, V, &g)) return SV_ERR_INVALID_ARG;
+    if (!target_logits || !draft_logits || !temperature || !log_norm || !row_status ||
+        (g.Ftot > 0 && (!out_tokens || !out_prob)))
+        return SV_ERR_INVALID_ARG;
+    if (!aligned(target_logits, 16) || !aligned(draft_logits, 16) || !aligned(temperature, 4) ||
+        !aligned(log_norm, 8) || !aligned(row_status, 4) || !aligned(out_tokens, 4) || !aligned(out_prob, 4))
+        return SV_ERR_MISALIGNED;
+    if (g.n_nz == 0) return SV_OK;
+    g.tgt = target_logits;
+    g.dft = draft_logits;
+    g.temperature = temperature;
+    g.log_norm = log_norm;
+    g.row_status = row_status;
+    g.out_tokens = out_tokens;
+    g.out_prob = out_prob;
+    const unsigned grid = (unsigned)((long long)B * g.n_nz);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dt == SV_DTYPE_BF16) sv::sv_topf<2><<<grid, sv::kTopfThreads, 0, st>>>(g);
+    else sv::sv_topf<4><<<grid, sv::kTopfThreads, 0, st>>>(g);
+    return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+extern "C" sv_status spec_verify_cache_lookup(const int32_t* out_tokens, const int32_t* out_n_accepted,
+                                              const int32_t* cache_tokens, const int32_t* fanout, int B,
+                                              int gamma, int32_t* out_slot, struct CUstream_st* stream)
+{
+    sv::TopfArgs g;
+    if (!fill_topf_args(fanout, B, gamma, 1, &g)) return SV_ERR_INVALID_ARG;
+    if (!out_tokens || !out_n_accepted || !out_slot || (g.Ftot > 0 && !cache_tokens)) return SV_ERR_INVALID_ARG;
+    if (!aligned(out_tokens, 4) || !aligned(out_n_accepted, 4) || !aligned(cache_tokens, 4) || !aligned(out_slot, 4))
+        return SV_ERR_MISALIGNED;
+    const unsigned grid = (unsigned)cdiv(B, 256);
+    sv::sv_cache_lookup<<<grid, 256, 0, (cudaStream_t)stream>>>(out_tokens, out_n_accepted, cache_tokens, g,
+                                                                  out_slot);
+    return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }

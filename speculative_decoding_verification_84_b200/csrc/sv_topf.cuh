@@ -1,0 +1,290 @@
+// sv_topf.cuh -- the speculation cache's side of an outcome [Speculative
+// Speculative Decoding, Metodologia 2, "Conceito Central" (the outcome is the
+// number accepted plus one more token; the cache holds speculations for likely
+// outcomes); Desafios 1 (a geometric fan-out over the accepted lengths) and 2
+// (the extra token after a rejection comes from the residual, whose mass
+// Saguaro sampling moves onto the cached top-F tokens)].
+//
+//   sv_topf          one CTA per (sequence b, outcome n with F_n > 0): the F_n
+//                    most probable tokens of the distribution the extra token is
+//                    drawn from after outcome n -- norm(max(0, p_n - q_n)) for
+//                    n < gamma (p_n when the residual mass is below 2^-18, as the
+//                    draw does), p_gamma for n = gamma, a point mass on the first
+//                    argmax of target row n when T = 0 -- with their
+//                    probabilities.  p and q come from the row log-normalisers
+//                    spec_verify returned, so this is one more pass over the draw
+//                    rows.  Each warp keeps the best F_n (weight, token) pairs of
+//                    its part of the rows in its lanes (lane i: the i-th best,
+//                    by weight, then smaller token); a candidate that beats lane
+//                    F_n - 1 is inserted by one ballot and one shuffle.  The CTA
+//                    then sorts the warps' 16 x 32 candidates (bitonic, shared
+//                    memory) and keeps the first F_n.
+//   sv_cache_lookup  one thread per sequence: the slot of outcome n's list that
+//                    holds the extra token spec_verify emitted, else -1.
+#pragma once
+
+#include "sv_common.cuh"
+
+namespace sv {
+
+constexpr int kTopfThreads = 512;
+constexpr int kTopfWarps = kTopfThreads / 32;
+
+struct TopfArgs {
+    const void* tgt;
+    const void* dft;
+    const float* temperature;
+    const double* log_norm;     // [B][2*gamma+1] from spec_verify
+    const int32_t* row_status;  // [B] from spec_verify
+    int32_t* out_tokens;        // [B][Ftot]
+    float* out_prob;            // [B][Ftot]
+    int F[SV_MAX_GAMMA + 1];    // slots per outcome
+    int off[SV_MAX_GAMMA + 2];  // first slot of each outcome
+    int Ftot, B, gamma, V;
+    int nz[SV_MAX_GAMMA + 1];   // the outcomes with F_n > 0, in order
+    int n_nz;
+};
+
+// (aw, av) ranks before (bw, bv): larger weight, then smaller token
+__device__ __forceinline__ bool ranks_before(float aw, int av, float bw, int bv)
+{
+    return aw > bw || (aw == bw && av < bv);
+}
+
+// Insert candidate (cw, cv), which ranks before lane F-1's pair, into the warp's
+// list (lane i holds the i-th best); the last pair drops out.
+__device__ __forceinline__ void list_insert(float& lw, int& lv, float cw, int cv, int F)
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned before = __ballot_sync(0xffffffffu, lane < F && ranks_before(lw, lv, cw, cv));
+    const int pos = __popc(before);
+    const float uw = __shfl_up_sync(0xffffffffu, lw, 1);
+    const int uv = __shfl_up_sync(0xffffffffu, lv, 1);
+    if (lane == pos) {
+        lw = cw;
+        lv = cv;
+    } else if (lane > pos) {
+        lw = uw;
+        lv = uv;
+    }
+}
+
+// Offer one candidate per lane (cw <= 0: none) to the warp's list, in lane order.
+__device__ __forceinline__ void list_offer(float& lw, int& lv, float& tw, int& tv, float cw, int cv, int F)
+{
+    const int lane = threadIdx.x & 31;
+    unsigned m = __ballot_sync(0xffffffffu, cw > 0.f && ranks_before(cw, cv, tw, tv));
+    while (m) {
+        const int src = __ffs(m) - 1;
+        const float w = __shfl_sync(0xffffffffu, cw, src);
+        const int v = __shfl_sync(0xffffffffu, cv, src);
+        list_insert(lw, lv, w, v, F);
+        tw = __shfl_sync(0xffffffffu, lw, F - 1);
+        tv = __shfl_sync(0xffffffffu, lv, F - 1);
+        m &= ~(1u << src);
+        m &= __ballot_sync(0xffffffffu, cw > 0.f && ranks_before(cw, cv, tw, tv));
+    }
+    (void)lane;
+}
+
+// The weights of row pair (t, d) at element i: max(0, p - q), or p (p_only),
+// p = 2^(l*k_hi + l*k_lo - mt) * ct with mt an integer and ct = 2^(mt - a2_t).
+struct TopfScale {
+    float khi, klo, mt, ct, md, cd;
+};
+
+__device__ __forceinline__ float topf_weight(const TopfScale& z, bool p_only, float lt, float ld)
+{
+    const float p = ex2(__fmaf_rn(lt, z.klo, __fmaf_rn(lt, z.khi, -z.mt))) * z.ct;
+    if (p_only) return p;
+    const float q = ex2(__fmaf_rn(ld, z.klo, __fmaf_rn(ld, z.khi, -z.md))) * z.cd;
+    return fmaxf(0.f, p - q);
+}
+
+// One pass over the CTA's rows: every warp's list of its part, the fp64 total of
+// the weights (block order), then the sorted CTA list in s_w / s_v.
+template <int ESZ>
+__device__ void topf_pass(const TopfArgs& g, const unsigned char* rt, const unsigned char* rd, bool p_only,
+                          const TopfScale& z, int F, float* s_w, int* s_v, double* s_sum, double& S)
+{
+    constexpr int VEC = 16 / ESZ;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int V = g.V;
+    const bool vec = ((size_t)V * ESZ) % 16 == 0;
+    float lw = -1.f, tw = -1.f;
+    int lv = 0x7fffffff, tv = 0x7fffffff;
+    double ls = 0.0;
+    if (vec) {
+        const int nv = V / VEC;
+        const int per = (nv + kTopfWarps - 1) / kTopfWarps;
+        const int w0 = min(nv, warp * per), w1 = min(nv, w0 + per);
+        for (int q0 = w0; q0 < w1; q0 += 32) {
+            const int q = q0 + lane;
+            const bool ok = q < w1;
+            float xt[VEC], xd[VEC];
+            unpack<ESZ>(ok ? __ldg(reinterpret_cast<const uint4*>(rt) + q) : make_uint4(0u, 0u, 0u, 0u), xt);
+            unpack<ESZ>((ok && !p_only) ? __ldg(reinterpret_cast<const uint4*>(rd) + q) : make_uint4(0u, 0u, 0u, 0u),
+                        xd);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                const float w = ok ? topf_weight(z, p_only, xt[e], xd[e]) : 0.f;
+                ls += (double)w;
+                list_offer(lw, lv, tw, tv, w, q * VEC + e, F);
+            }
+        }
+    } else {
+        const int per = (V + kTopfWarps - 1) / kTopfWarps;
+        const int e0 = min(V, warp * per), e1 = min(V, e0 + per);
+        for (int i0 = e0; i0 < e1; i0 += 32) {
+            const int i = i0 + lane;
+            const bool ok = i < e1;
+            const float lt = ok ? load_logit<ESZ>(rt, (size_t)i) : 0.f;
+            const float ld = (ok && !p_only) ? load_logit<ESZ>(rd, (size_t)i) : 0.f;
+            const float w = ok ? topf_weight(z, p_only, lt, ld) : 0.f;
+            ls += (double)w;
+            list_offer(lw, lv, tw, tv, w, i, F);
+        }
+    }
+    // the total, in a fixed order: lanes, then warps
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane == 0) s_sum[warp] = ls;
+    s_w[tid] = lane < F ? lw : -1.f;
+    s_v[tid] = lane < F ? lv : 0x7fffffff;
+    __syncthreads();
+    S = 0.0;
+    for (int k = 0; k < kTopfWarps; ++k) S += s_sum[k];
+    // bitonic sort of the kTopfThreads candidates, best first
+    for (int k = 2; k <= kTopfThreads; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const int ixj = tid ^ j;
+            if (ixj > tid) {
+                const float aw = s_w[tid], bw = s_w[ixj];
+                const int av = s_v[tid], bv = s_v[ixj];
+                const bool up = (tid & k) == 0;  // this block ends best first
+                const bool swap = up ? ranks_before(bw, bv, aw, av) : ranks_before(aw, av, bw, bv);
+                if (swap) {
+                    s_w[tid] = bw;
+                    s_v[tid] = bv;
+                    s_w[ixj] = aw;
+                    s_v[ixj] = av;
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+template <int ESZ>
+__global__ void __launch_bounds__(kTopfThreads, 1) sv_topf(const __grid_constant__ TopfArgs g)
+{
+    __shared__ float s_w[kTopfThreads];
+    __shared__ int s_v[kTopfThreads];
+    __shared__ double s_sum[kTopfWarps];
+    __shared__ int s_arg;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int b = blockIdx.x / g.n_nz;
+    const int n = g.nz[blockIdx.x - b * g.n_nz];
+    const int gamma = g.gamma, R = 2 * gamma + 1, F = g.F[n];
+    int32_t* ot = g.out_tokens + (size_t)b * g.Ftot + g.off[n];
+    float* op = g.out_prob + (size_t)b * g.Ftot + g.off[n];
+    const float T = __ldg(g.temperature + b);
+    const int st = __ldg(g.row_status + b);
+    // a sequence with an invalid temperature or a bad row has no distributions
+    bool bad = (st & (SV_ROW_BAD_TEMPERATURE | SV_ROW_BAD_LOGITS)) != 0 || !temperature_ok(T);
+    const double* ln = g.log_norm + (size_t)b * R;
+    if (!bad && T != 0.f)
+        for (int r = 0; r < R; ++r) bad = bad || !isfinite(__ldg(ln + r));
+    if (bad) {
+        for (int s = tid; s < F; s += kTopfThreads) {
+            ot[s] = -1;
+            op[s] = 0.f;
+        }
+        return;
+    }
+    const size_t rowb = (size_t)g.V * ESZ;
+    const unsigned char* rt = static_cast<const unsigned char*>(g.tgt) + ((size_t)b * (gamma + 1) + n) * rowb;
+    if (T == 0.f) {
+        // a point mass on the first argmax of target row n
+        Amax A{-INFINITY, 0x7fffffff, 0};
+        for (int i = tid; i < g.V; i += kTopfThreads) amax_add(A, load_logit<ESZ>(rt, (size_t)i), i);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, A.best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, A.idx, o);
+            const int on = __shfl_xor_sync(0xffffffffu, A.nan, o);
+            amax_merge(A, ob, oi, on);
+        }
+        // the warps' maxima, merged in warp order (each warp saw interleaved indices,
+        // so the merge keeps the best value's smallest index)
+        if (lane == 0) {
+            s_w[tid >> 5] = A.best;
+            s_v[tid >> 5] = A.idx;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            Amax B{-INFINITY, 0x7fffffff, 0};
+            for (int k = 0; k < kTopfWarps; ++k) amax_merge(B, s_w[k], s_v[k], 0);
+            s_arg = B.idx;
+        }
+        __syncthreads();
+        for (int s = tid; s < F; s += kTopfThreads) {
+            ot[s] = s == 0 ? s_arg : -1;
+            op[s] = s == 0 ? 1.f : 0.f;
+        }
+        return;
+    }
+    const unsigned char* rd = n < gamma ? static_cast<const unsigned char*>(g.dft) + ((size_t)b * gamma + n) * rowb
+                                        : rt;
+    TopfScale z;
+    split_k(T, &z.khi, &z.klo);
+    {
+        // p_v = 2^(l_v*k - a2) with a2 = lse*log2(e): the integer part of a2 is the
+        // offset, the rest a factor in [1, 2)
+        const double a2t = __ldg(ln + n) * kLog2e;
+        const double ft = floor(a2t);
+        z.mt = (float)ft;
+        z.ct = (float)exp2(ft - a2t);
+        z.md = 0.f;
+        z.cd = 0.f;
+        if (n < gamma) {
+            const double a2d = __ldg(ln + gamma + 1 + n) * kLog2e;
+            const double fd = floor(a2d);
+            z.md = (float)fd;
+            z.cd = (float)exp2(fd - a2d);
+        }
+    }
+    double S;
+    bool p_only = (n == gamma);
+    topf_pass<ESZ>(g, rt, rd, p_only, z, F, s_w, s_v, s_sum, S);
+    if (!p_only && !(S >= kResidualMin)) {
+        // the residual vanished (below kResidualMin): p_n, as the draw
+        __syncthreads();
+        topf_pass<ESZ>(g, rt, rd, true, z, F, s_w, s_v, s_sum, S);
+    }
+    for (int s = tid; s < F; s += kTopfThreads) {
+        const float w = s_w[s];
+        ot[s] = w > 0.f ? s_v[s] : -1;
+        op[s] = w > 0.f ? (float)((double)w / S) : 0.f;
+    }
+}
+
+// The slot of each sequence's outcome (n, extra token) in its cache, else -1.
+__global__ void sv_cache_lookup(const int32_t* __restrict__ out_tokens, const int32_t* __restrict__ out_n,
+                                const int32_t* __restrict__ cache, const __grid_constant__ TopfArgs g,
+                                int32_t* __restrict__ out_slot)
+{
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= g.B) return;
+    int slot = -1;
+    const int n = __ldg(out_n + b);
+    if (n >= 0 && n <= g.gamma) {
+        const int x = __ldg(out_tokens + (size_t)b * (g.gamma + 1) + n);
+        if (x >= 0)
+            for (int s = g.off[n]; s < g.off[n + 1] && slot < 0; ++s)
+                if (__ldg(cache + (size_t)b * g.Ftot + s) == x) slot = s;
+    }
+    out_slot[b] = slot;
+}
+
+}  // namespace sv

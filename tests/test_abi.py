@@ -85,3 +85,19 @@ def test_host_validation_before_launch(lib):
     assert lib.spec_verify(*small) == 4
     for s in range(6):
         assert lib.spec_verify_status_string(s)
+
+
+def test_fanout_host_matches_oracle(lib):
+    """spec_verify_fanout runs on the host: it must allocate the slots exactly as
+    the oracle's geometric rule (pinned in topf_pins.check_fanout_closed_forms)."""
+    import numpy as np
+    import oracle
+    for alpha in (0.0, 0.1, 0.33, 0.5, 0.7, 0.95, 1.0):
+        for gamma in (1, 4, 5, 8, 32):
+            for budget in (0, 1, 3, 16, 64, 255):
+                got = binding.fanout(alpha, gamma, budget)
+                assert (got == oracle.fanout(alpha, gamma, budget)).all(), (alpha, gamma, budget)
+    F = np.empty(3, np.int32)
+    assert lib.spec_verify_fanout(1.5, 2, 4, F.ctypes.data) != 0
+    assert lib.spec_verify_fanout(0.5, 0, 4, F.ctypes.data) != 0
+    assert lib.spec_verify_fanout(0.5, 2, -1, F.ctypes.data) != 0
