@@ -322,6 +322,90 @@ def config_line(c, peak, peak_kind, hot=False, budget_ms=20.0):
     }
 
 
+def cache_row_line(w, dev, lib, binding, peak, peak_kind, budget_ms=20.0):
+    """The speculation-cache row on one workload: spec_verify_topf with the
+    geometric fan-out of a 64-slot budget at acceptance rate 0.7 (then at most 32
+    per outcome), and spec_verify_cache_lookup; each timed as CUDA graph replays
+    over the input copies, after one untimed spec_verify per copy supplied the
+    normalisers and row status."""
+    import torch
+    c = Caller(w, dev, lib, binding)
+    F = np.minimum(binding.fanout(0.7, c.gamma, 64), binding.MAX_TOPF).astype(np.int32)
+    Ft = int(F.sum())
+    ln = [torch.empty((c.B, 2 * c.gamma + 1), dtype=torch.float64, device=dev) for _ in range(c.n_copies)]
+    st = [torch.empty((c.B,), dtype=torch.int32, device=dev) for _ in range(c.n_copies)]
+    toks = [torch.empty((c.B, c.gamma + 1), dtype=torch.int32, device=dev) for _ in range(c.n_copies)]
+    nacc = [torch.empty((c.B,), dtype=torch.int32, device=dev) for _ in range(c.n_copies)]
+    with torch.cuda.stream(c.stream):
+        for i in range(c.n_copies):
+            d = c.sets[i]
+            rc = lib.spec_verify(d["target"].data_ptr(), d["draft"].data_ptr(), c.dt_code, d["draft_tokens"].data_ptr(),
+                                 d["temperature"].data_ptr(), d["u_accept"].data_ptr(), d["u_resample"].data_ptr(),
+                                 toks[i].data_ptr(), nacc[i].data_ptr(), c.B, c.gamma, c.V, c.wspace.data_ptr(),
+                                 c.wsz, ln[i].data_ptr(), st[i].data_ptr(), c.stream.cuda_stream)
+            if rc != 0:
+                raise RuntimeError(binding.status_string(rc))
+    otok = torch.empty((c.B, Ft), dtype=torch.int32, device=dev)
+    oprob = torch.empty((c.B, Ft), dtype=torch.float32, device=dev)
+    slot = torch.empty((c.B,), dtype=torch.int32, device=dev)
+
+    def topf(i):
+        d = c.sets[i % c.n_copies]
+        j = i % c.n_copies
+        rc = lib.spec_verify_topf(d["target"].data_ptr(), d["draft"].data_ptr(), c.dt_code, d["temperature"].data_ptr(),
+                                  ln[j].data_ptr(), st[j].data_ptr(), F.ctypes.data, c.B, c.gamma, c.V,
+                                  otok.data_ptr(), oprob.data_ptr(), c.stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(binding.status_string(rc))
+
+    def lookup(i):
+        j = i % c.n_copies
+        rc = lib.spec_verify_cache_lookup(toks[j].data_ptr(), nacc[j].data_ptr(), otok.data_ptr(), F.ctypes.data,
+                                          c.B, c.gamma, slot.data_ptr(), c.stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(binding.status_string(rc))
+
+    def graph_time(fn, k):
+        n = c.n_copies * max(1, -(-16 // c.n_copies))
+        g = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=c.stream):
+            for i in range(n):
+                fn(i)
+        reps = max(3, -(-k // n))
+        with torch.cuda.stream(c.stream):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(c.stream)
+        with torch.cuda.stream(c.stream):
+            for _ in range(reps):
+                g.replay()
+        e1.record(c.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * n)
+
+    with torch.cuda.stream(c.stream):
+        for i in range(4):
+            topf(i)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(c.stream):
+        topf(0)
+    torch.cuda.synchronize()
+    probe = (time.perf_counter() - t0) * 1e3
+    k = int(max(20, min(2000, budget_ms / max(probe, 1e-3))))
+    ms_topf = graph_time(topf, k)
+    ms_lookup = graph_time(lookup, k)
+    rows = sum(int(F[n] > 0) * (2 if n < c.gamma else 1) for n in range(c.gamma + 1))
+    alg = c.B * rows * c.V * c.esz
+    gbs = alg / (ms_topf / 1e3) / 1e9
+    return {"workload": w.name, "fanout": F.tolist(), "slots": Ft, "us_per_call_topf": 1e3 * ms_topf,
+            "us_per_call_lookup": 1e3 * ms_lookup, "algorithmic_bytes_topf": alg,
+            "note": "bytes: the draw rows of every outcome with slots, read once", "hbm_gbs": gbs,
+            "frac_of_peak": gbs / peak, "peak_source": peak_kind}
+
+
 def run_ours(args):
     import torch
     ws, rank, local = dist_env()
@@ -438,6 +522,8 @@ def run_ours(args):
                 del cc
             del wc
             torch.cuda.empty_cache()
+        per_config["cache_row_c3"] = cache_row_line(W.make_workload(WORKLOAD), dev, lib, binding, peak, peak_kind)
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

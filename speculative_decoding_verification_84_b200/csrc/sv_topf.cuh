@@ -29,6 +29,7 @@ namespace sv {
 
 constexpr int kTopfThreads = 512;
 constexpr int kTopfWarps = kTopfThreads / 32;
+constexpr int kTopfBatch = 4;  // 16-byte vectors per lane and row loaded before any is used
 
 struct TopfArgs {
     const void* tgt;
@@ -69,22 +70,48 @@ __device__ __forceinline__ void list_insert(float& lw, int& lv, float cw, int cv
     }
 }
 
-// Offer one candidate per lane (cw <= 0: none) to the warp's list, in lane order.
-__device__ __forceinline__ void list_offer(float& lw, int& lv, float& tw, int& tv, float cw, int cv, int F)
+// The lane's candidates in w[0..VEC) (tokens i0 + e) that rank before the list's
+// last pair, as a bit mask.
+template <int VEC>
+__device__ __forceinline__ unsigned qualifying(const float (&w)[VEC], int i0, float tw, int tv, float bar)
+{
+    unsigned qm = 0;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e)
+        if (w[e] > 0.f && w[e] >= bar && ranks_before(w[e], i0 + e, tw, tv)) qm |= 1u << e;
+    return qm;
+}
+
+// Insert every qualifying candidate of the warp, one per round: the lowest lane
+// that has one offers its first; then every lane re-tests its own against the
+// raised bar.  The rounds are as many as the insertions (the final list does not
+// depend on their order: the ranking is a total order).
+template <int VEC>
+__device__ __forceinline__ void list_offer_vec(float& lw, int& lv, float& tw, int& tv, const float (&w)[VEC],
+                                               int i0, int F, unsigned qm, int* s_bar)
 {
     const int lane = threadIdx.x & 31;
-    unsigned m = __ballot_sync(0xffffffffu, cw > 0.f && ranks_before(cw, cv, tw, tv));
+    unsigned m = __ballot_sync(0xffffffffu, qm != 0);
+    if (!m) return;
     while (m) {
         const int src = __ffs(m) - 1;
-        const float w = __shfl_sync(0xffffffffu, cw, src);
-        const int v = __shfl_sync(0xffffffffu, cv, src);
-        list_insert(lw, lv, w, v, F);
+        const int e0 = qm ? __ffs(qm) - 1 : 0;
+        float cw = w[0];
+#pragma unroll
+        for (int e = 1; e < VEC; ++e)
+            if (e == e0) cw = w[e];
+        cw = __shfl_sync(0xffffffffu, cw, src);
+        const int cv = __shfl_sync(0xffffffffu, i0 + e0, src);
+        list_insert(lw, lv, cw, cv, F);
         tw = __shfl_sync(0xffffffffu, lw, F - 1);
         tv = __shfl_sync(0xffffffffu, lv, F - 1);
-        m &= ~(1u << src);
-        m &= __ballot_sync(0xffffffffu, cw > 0.f && ranks_before(cw, cv, tw, tv));
+        if (lane == src) qm &= ~(1u << e0);
+        qm &= qualifying<VEC>(w, i0, tw, tv, 0.f);
+        m = __ballot_sync(0xffffffffu, qm != 0);
     }
-    (void)lane;
+    // a full list's last weight bounds the CTA's F-th weight from below: publish it
+    // (weights are >= 0, so their bit patterns order as integers)
+    if (lane == 0 && tw > 0.f) atomicMax(s_bar, __float_as_int(tw));
 }
 
 // The weights of row pair (t, d) at element i: max(0, p - q), or p (p_only),
@@ -101,11 +128,19 @@ __device__ __forceinline__ float topf_weight(const TopfScale& z, bool p_only, fl
     return fmaxf(0.f, p - q);
 }
 
+// The sum of a vector's weights, as a short tree (4 or 8 elements).
+template <int N>
+__device__ __forceinline__ float tree8_any(const float (&w)[N])
+{
+    if (N == 8) return ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+    return (w[0] + w[1]) + (w[2] + w[3]);
+}
+
 // One pass over the CTA's rows: every warp's list of its part, the fp64 total of
 // the weights (block order), then the sorted CTA list in s_w / s_v.
 template <int ESZ>
 __device__ void topf_pass(const TopfArgs& g, const unsigned char* rt, const unsigned char* rd, bool p_only,
-                          const TopfScale& z, int F, float* s_w, int* s_v, double* s_sum, double& S)
+                          const TopfScale& z, int F, float* s_w, int* s_v, double* s_sum, int* s_bar, double& S)
 {
     constexpr int VEC = 16 / ESZ;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -118,18 +153,31 @@ __device__ void topf_pass(const TopfArgs& g, const unsigned char* rt, const unsi
         const int nv = V / VEC;
         const int per = (nv + kTopfWarps - 1) / kTopfWarps;
         const int w0 = min(nv, warp * per), w1 = min(nv, w0 + per);
-        for (int q0 = w0; q0 < w1; q0 += 32) {
-            const int q = q0 + lane;
+        // kTopfBatch vectors per lane and row in flight at once
+        for (int q0 = w0; q0 < w1; q0 += 32 * kTopfBatch) {
+            uint4 vt[kTopfBatch], vd[kTopfBatch];
+#pragma unroll
+            for (int u = 0; u < kTopfBatch; ++u) {
+                const int q = q0 + u * 32 + lane;
+                vt[u] = q < w1 ? __ldg(reinterpret_cast<const uint4*>(rt) + q) : make_uint4(0u, 0u, 0u, 0u);
+                vd[u] = (q < w1 && !p_only) ? __ldg(reinterpret_cast<const uint4*>(rd) + q) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kTopfBatch; ++u) {
+            const int q = q0 + u * 32 + lane;
             const bool ok = q < w1;
             float xt[VEC], xd[VEC];
-            unpack<ESZ>(ok ? __ldg(reinterpret_cast<const uint4*>(rt) + q) : make_uint4(0u, 0u, 0u, 0u), xt);
-            unpack<ESZ>((ok && !p_only) ? __ldg(reinterpret_cast<const uint4*>(rd) + q) : make_uint4(0u, 0u, 0u, 0u),
-                        xd);
+            unpack<ESZ>(vt[u], xt);
+            unpack<ESZ>(vd[u], xd);
+            float w[VEC];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                const float w = ok ? topf_weight(z, p_only, xt[e], xd[e]) : 0.f;
-                ls += (double)w;
-                list_offer(lw, lv, tw, tv, w, q * VEC + e, F);
+            for (int e = 0; e < VEC; ++e) w[e] = ok ? topf_weight(z, p_only, xt[e], xd[e]) : 0.f;
+            ls += (double)tree8_any<VEC>(w);
+            // one vote per vector; rounds only for the candidates that beat the list
+            // and are not below another warp's published F-th weight (F pairs of that
+            // warp outrank them)
+            const float bar = __int_as_float(*reinterpret_cast<volatile int*>(s_bar));
+            list_offer_vec<VEC>(lw, lv, tw, tv, w, q * VEC, F, qualifying<VEC>(w, q * VEC, tw, tv, bar), s_bar);
             }
         }
     } else {
@@ -140,9 +188,10 @@ __device__ void topf_pass(const TopfArgs& g, const unsigned char* rt, const unsi
             const bool ok = i < e1;
             const float lt = ok ? load_logit<ESZ>(rt, (size_t)i) : 0.f;
             const float ld = (ok && !p_only) ? load_logit<ESZ>(rd, (size_t)i) : 0.f;
-            const float w = ok ? topf_weight(z, p_only, lt, ld) : 0.f;
-            ls += (double)w;
-            list_offer(lw, lv, tw, tv, w, i, F);
+            const float w1[1] = {ok ? topf_weight(z, p_only, lt, ld) : 0.f};
+            ls += (double)w1[0];
+            const float bar = __int_as_float(*reinterpret_cast<volatile int*>(s_bar));
+            list_offer_vec<1>(lw, lv, tw, tv, w1, i, F, qualifying<1>(w1, i, tw, tv, bar), s_bar);
         }
     }
     // the total, in a fixed order: lanes, then warps
@@ -182,6 +231,7 @@ __global__ void __launch_bounds__(kTopfThreads, 1) sv_topf(const __grid_constant
     __shared__ int s_v[kTopfThreads];
     __shared__ double s_sum[kTopfWarps];
     __shared__ int s_arg;
+    __shared__ int s_bar[1];  // bits of the largest F-th weight any warp has published
     const int tid = threadIdx.x, lane = tid & 31;
     const int b = blockIdx.x / g.n_nz;
     const int n = g.nz[blockIdx.x - b * g.n_nz];
@@ -256,11 +306,15 @@ __global__ void __launch_bounds__(kTopfThreads, 1) sv_topf(const __grid_constant
     }
     double S;
     bool p_only = (n == gamma);
-    topf_pass<ESZ>(g, rt, rd, p_only, z, F, s_w, s_v, s_sum, S);
+    if (tid == 0) *s_bar = 0;
+    __syncthreads();
+    topf_pass<ESZ>(g, rt, rd, p_only, z, F, s_w, s_v, s_sum, s_bar, S);
     if (!p_only && !(S >= kResidualMin)) {
         // the residual vanished (below kResidualMin): p_n, as the draw
         __syncthreads();
-        topf_pass<ESZ>(g, rt, rd, true, z, F, s_w, s_v, s_sum, S);
+        if (tid == 0) *s_bar = 0;
+        __syncthreads();
+        topf_pass<ESZ>(g, rt, rd, true, z, F, s_w, s_v, s_sum, s_bar, S);
     }
     for (int s = tid; s < F; s += kTopfThreads) {
         const float w = s_w[s];
