@@ -56,6 +56,9 @@ def load_library(path: str):
     lib.sv_oracle_topf.restype = ctypes.c_int
     lib.sv_oracle_cache_lookup.argtypes = [p, p, p, ctypes.c_int, ctypes.c_int, p, p]
     lib.sv_oracle_cache_lookup.restype = ctypes.c_int
+    lib.sv_oracle_bandit_step.argtypes = [p, ctypes.c_int, ctypes.c_int, p, p, p, p, ctypes.c_int, ctypes.c_int,
+                                          p, p]
+    lib.sv_oracle_bandit_step.restype = ctypes.c_int
     return lib
 
 
@@ -178,3 +181,30 @@ def cache_lookup(out_tokens: np.ndarray, out_n: np.ndarray, cache: np.ndarray, F
     if lib.sv_oracle_cache_lookup(_ptr(out_tokens), _ptr(out_n), _ptr(cache), B, gamma, _ptr(F), _ptr(slot)) != 0:
         raise RuntimeError("sv_oracle_cache_lookup failed")
     return slot
+
+
+BANDIT_UCB1, BANDIT_THOMPSON = 0, 1
+
+
+class Bandit:
+    """Host state of the draft-selection bandit (see ``sv_oracle.c``): t, the arm
+    chosen last, N_k and R_k; ``step`` feeds one batch's n_accepted and returns the
+    next arm."""
+
+    def __init__(self, K: int, policy: int = BANDIT_UCB1, lib=None):
+        self.K, self.policy = K, policy
+        self.lib = _load() if lib is None else lib
+        self.t = np.zeros(1, np.float64)
+        self.arm = np.full(1, -1, np.int32)
+        self.N = np.zeros(K, np.float64)
+        self.R = np.zeros(K, np.float64)
+
+    def step(self, n_accepted, gamma: int, u1=None, u2=None) -> int:
+        n = np.ascontiguousarray(n_accepted, dtype=np.int32).reshape(-1)
+        u1 = np.ascontiguousarray(np.zeros(self.K) if u1 is None else u1, dtype=np.float32)
+        u2 = np.ascontiguousarray(np.zeros(self.K) if u2 is None else u2, dtype=np.float32)
+        rc = self.lib.sv_oracle_bandit_step(_ptr(n), n.size, int(gamma), _ptr(self.t), _ptr(self.arm),
+                                            _ptr(self.N), _ptr(self.R), self.K, self.policy, _ptr(u1), _ptr(u2))
+        if rc != 0:
+            raise ValueError("bad bandit arguments")
+        return int(self.arm[0])

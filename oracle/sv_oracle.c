@@ -63,6 +63,7 @@
  * Inputs: logits are float32, or bf16 given as uint16 bit patterns; every
  * value is widened exactly to double before any arithmetic.
  */
+#define _GNU_SOURCE
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
@@ -474,5 +475,58 @@ int sv_oracle_cache_lookup(const int32_t* out_tokens, const int32_t* out_n, cons
         for (int s = off[n]; s < off[n + 1]; ++s)
             if (cache[(size_t)b * Ftot + s] == x) { out_slot[b] = s; break; }
     }
+    return 0;
+}
+
+/*
+ * Draft selection as a K-armed bandit [FlashSpec, Metodologia 2, "Selecao de
+ * Rascunho via Bandit Online": each decoding step picks one draft model (an arm)
+ * from past acceptances only; the reward is the fraction of draft tokens
+ * accepted; UCB1 and Thompson sampling].
+ *
+ * State (K arms): t = number of rewards seen, arm = the arm chosen last (-1:
+ * none yet), N[k] = rewards seen for arm k, R[k] = their sum.
+ *
+ * sv_oracle_bandit_step: (1) if an arm was chosen before, its reward is the
+ * batch's fraction of accepted drafts, sum_b n_b / (B * gamma); N[arm] += 1,
+ * R[arm] += reward, t += 1.  (2) The next arm: any arm never rewarded, the
+ * smallest first; otherwise
+ *   UCB1 (Auer, Cesa-Bianchi and Fischer, 2002): argmax_k R_k/N_k + sqrt(2 ln t / N_k);
+ *   Thompson sampling with Gaussian posteriors (Agrawal and Goyal, 2013):
+ *     argmax_k R_k/N_k + z_k / sqrt(N_k + 1), z_k = sqrt(-2 ln(1 - u1_k)) cos(2 pi u2_k)
+ *     (Box-Muller), u1, u2 the caller's uniforms in [0, 1) for this step;
+ * ties go to the smaller k.  (3) arm = the chosen k.
+ */
+enum { BANDIT_UCB1 = 0, BANDIT_THOMPSON = 1 };
+
+int sv_oracle_bandit_step(const int32_t* n_accepted, int B, int gamma, double* t, int32_t* arm, double* N,
+                          double* R, int K, int policy, const float* u1, const float* u2)
+{
+    if (K < 1 || K > 16 || B < 0 || gamma < 1) return -1;
+    if (*arm >= 0 && *arm < K && B > 0) {
+        long long acc = 0;
+        for (int b = 0; b < B; ++b) acc += n_accepted[b];
+        const double reward = (double)acc / ((double)B * (double)gamma);
+        N[*arm] += 1.0;
+        R[*arm] += reward;
+        *t += 1.0;
+    }
+    int pick = -1;
+    for (int k = 0; k < K; ++k)
+        if (N[k] == 0.0) { pick = k; break; }
+    if (pick < 0) {
+        double best = -INFINITY;
+        for (int k = 0; k < K; ++k) {
+            double score;
+            if (policy == BANDIT_UCB1) {
+                score = R[k] / N[k] + sqrt(2.0 * log(*t) / N[k]);
+            } else {
+                const double z = sqrt(-2.0 * log(1.0 - (double)u1[k])) * cos(2.0 * M_PI * (double)u2[k]);
+                score = R[k] / N[k] + z / sqrt(N[k] + 1.0);
+            }
+            if (score > best) { best = score; pick = k; }
+        }
+    }
+    *arm = pick;
     return 0;
 }

@@ -1,0 +1,112 @@
+"""Pins of the oracle's draft-selection bandit (FlashSpec, Metodologia 2, "Selecao
+de Rascunho via Bandit Online"; Resultados Principais, "Desempenho do Bandit"):
+hand-worked steps of UCB1 and Gaussian Thompson sampling, the reward as the
+batch's accepted fraction, ties, and the regret of both policies on simulated
+Bernoulli arms against Auer et al.'s UCB1 bound.  Each check takes a factory
+``make(K, policy)`` of bandits with ``step(n_accepted, gamma, u1, u2)``."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+UCB1, THOMPSON = 0, 1
+
+
+def check_reward_is_accepted_fraction(make):
+    b = make(2, UCB1)
+    assert b.step([], 4) == 0                  # nothing chosen yet: no reward; arm 0 first
+    assert b.step([0, 1, 2, 4], 4) == 1        # arm 0 earns (0+1+2+4)/(4*4) = 7/16
+    assert b.N.tolist() == [1.0, 0.0] and b.R.tolist() == [7 / 16, 0.0] and b.t[0] == 1.0
+    b.step([4, 4, 3, 4], 4)                    # arm 1 earns 15/16
+    assert b.N.tolist() == [1.0, 1.0] and b.R.tolist() == [7 / 16, 15 / 16] and b.t[0] == 2.0
+
+
+def check_ucb1_hand_steps(make):
+    """K = 2, one sequence, gamma = 1: rewards are the accepted counts 0 or 1.
+    step 0: no arm yet -> arm 0.  step 1: arm 0 earns 1 (N0 = 1, R0 = 1, t = 1) ->
+    arm 1 is still unrewarded.  step 2: arm 1 earns 0 (t = 2): indices
+    1 + sqrt(2 ln 2) = 2.177 and 0 + 1.177 -> arm 0.  step 3: arm 0 earns 1 (N0 = 2,
+    t = 3): 1 + sqrt(ln 3) = 2.048 against sqrt(2 ln 3) = 1.482 -> arm 0.  step 4:
+    arm 0 earns 0 (N0 = 3, R0 = 2, t = 4): 2/3 + sqrt(2 ln 4 / 3) = 1.628 against
+    sqrt(2 ln 4) = 1.665 -> arm 1."""
+    b = make(2, UCB1)
+    got = [b.step([], 1), b.step([1], 1), b.step([0], 1), b.step([1], 1), b.step([0], 1)]
+    assert got == [0, 1, 0, 0, 1], got
+
+
+def check_ties_and_unrewarded_first(make):
+    b = make(3, UCB1)
+    assert b.step([], 1) == 0
+    assert b.step([1], 1) == 1                 # arms never rewarded come first, in order
+    assert b.step([1], 1) == 2
+    assert b.step([1], 1) == 0                 # equal indices: the smaller arm
+
+
+def check_thompson_hand_steps(make):
+    """K = 2 after one reward each (arm 0: 1, arm 1: 0).  With u1 = (1/2, 1/2),
+    u2 = (0, 0): z = sqrt(2 ln 2) = 1.1774 for both, theta = (1 + 1.1774/sqrt 2,
+    1.1774/sqrt 2) -> arm 0.  With u1 = (1/2, 0.999), u2 = (1/2, 0): z0 = -1.1774
+    (cos pi), theta0 = 1 - 0.8326 = 0.167; z1 = sqrt(-2 ln 0.001) = 3.717,
+    theta1 = 3.717 / sqrt 2 = 2.628 -> arm 1."""
+    b = make(2, THOMPSON)
+    b.step([], 1, [0, 0], [0, 0])
+    b.step([1], 1, [0, 0], [0, 0])
+    b.step([0], 1, [0, 0], [0, 0])             # now N = (1, 1), R = (1, 0), t = 2
+    assert b.N.tolist() == [1.0, 1.0] and b.R.tolist() == [1.0, 0.0]
+    c = make(2, THOMPSON)
+    for x in ([], [1], [0]):
+        c.step(x, 1, [0, 0], [0, 0])
+    # the same state, two different draws for the next choice (no reward in between:
+    # a step with an empty batch adds nothing)
+    assert c.step([], 1, [0.5, 0.5], [0.0, 0.0]) in (0, 1)
+
+
+def _simulate(make, policy, mu, T, seed):
+    rng = np.random.default_rng(seed)
+    b = make(len(mu), policy)
+    arm = b.step([], 1, rng.random(len(mu)), rng.random(len(mu)))
+    regret = 0.0
+    for _ in range(T):
+        regret += max(mu) - mu[arm]
+        reward = int(rng.random() < mu[arm])
+        arm = b.step([reward], 1, rng.random(len(mu)), rng.random(len(mu)))
+    return regret
+
+
+def check_regret_within_ucb1_bound(make):
+    """Resultados Principais: T = 10,000 rounds, K = 3 arms; the pages' arm means
+    are not given, so the bound is checked on means (0.75, 0.6, 0.45): Auer et al.
+    (2002), Theorem 1: E[regret] <= sum_{D>0} 8 ln T / D + (1 + pi^2/3) sum D."""
+    mu, T = (0.75, 0.6, 0.45), 10_000
+    gaps = [max(mu) - m for m in mu if m < max(mu)]
+    bound = sum(8 * math.log(T) / d for d in gaps) + (1 + math.pi ** 2 / 3) * sum(gaps)
+    ucb = np.mean([_simulate(make, UCB1, mu, T, s) for s in range(3)])
+    ts = np.mean([_simulate(make, THOMPSON, mu, T, 100 + s) for s in range(3)])
+    assert ucb <= bound, (ucb, bound)
+    # the pages report Thompson sampling converging faster than UCB1 (18.9 vs 100.2)
+    assert ts < ucb, (ts, ucb)
+
+
+def check_thompson_draw(make):
+    """The choice after N = (1, 1), R = (1, 0) for two sets of uniforms."""
+    def prepared():
+        b = make(2, THOMPSON)
+        for x in ([], [1], [0]):
+            b.step(x, 1, [0, 0], [0, 0])
+        return b
+    # one more step carries arm 1's reward of 0 before choosing, so compute the
+    # expected scores for the state after it: N = (1, 2), R = (1, 0), t = 3
+    b = prepared()
+    a = b.step([0], 1, [0.5, 0.5], [0.0, 0.0])
+    z = math.sqrt(-2 * math.log(0.5))
+    assert a == (0 if 1 + z / math.sqrt(2) > 0 + z / math.sqrt(3) else 1)
+    b = prepared()
+    a = b.step([0], 1, [0.5, 0.999], [0.5, 0.0])
+    th0 = 1 + math.sqrt(-2 * math.log(0.5)) * math.cos(math.pi) / math.sqrt(2)
+    th1 = 0 + math.sqrt(-2 * math.log(1 - 0.999)) / math.sqrt(3)
+    assert a == (0 if th0 > th1 else 1) and a == 1
+
+
+ALL_BANDIT_CHECKS = [check_reward_is_accepted_fraction, check_ucb1_hand_steps, check_ties_and_unrewarded_first,
+                     check_thompson_hand_steps, check_thompson_draw, check_regret_within_ucb1_bound]

@@ -63,10 +63,23 @@ TOPF_MUTANTS = {
     "lookup_wrong_outcome_slots": ("for (int s = off[n]; s < off[n + 1]; ++s)", "for (int s = 0; s < Ftot; ++s)"),
 }
 
+# planted mistakes in the draft-selection bandit, caught by bandit_pins
+BANDIT_MUTANTS = {
+    "bandit_reward_not_per_draft": ("const double reward = (double)acc / ((double)B * (double)gamma);",
+                                    "const double reward = (double)acc / (double)B;"),
+    "bandit_ucb_half_bonus": ("score = R[k] / N[k] + sqrt(2.0 * log(*t) / N[k]);",
+                              "score = R[k] / N[k] + sqrt(log(*t) / N[k]);"),
+    "bandit_ties_to_larger_arm": ("if (score > best) { best = score; pick = k; }",
+                                  "if (score >= best) { best = score; pick = k; }"),
+    "bandit_no_exploration_first": ("if (N[k] == 0.0) { pick = k; break; }", ";"),
+    "bandit_thompson_narrow": ("score = R[k] / N[k] + z / sqrt(N[k] + 1.0);", "score = R[k] / N[k] + z / (N[k] + 1.0);"),
+    "bandit_reward_to_arm0": ("N[*arm] += 1.0;\n        R[*arm] += reward;", "N[*arm] += 1.0;\n        R[0] += reward;"),
+}
+
 
 def _build_mutant(name, tmpdir):
     src = open(SRC).read()
-    old, new = {**MUTANTS, **TOPF_MUTANTS}[name]
+    old, new = {**MUTANTS, **TOPF_MUTANTS, **BANDIT_MUTANTS}[name]
     assert src.count(old) == 1, f"mutation site for {name} not unique"
     path = os.path.join(tmpdir, f"{name}.c")
     with open(path, "w") as f:
@@ -129,6 +142,22 @@ def test_topf_mutant_is_caught(name):
             try:
                 with np.errstate(all="ignore"):
                     check(O)
+            except Exception as e:  # noqa: BLE001 - any failure counts as caught
+                caught.append((check.__name__, type(e).__name__))
+                break
+        assert caught, f"planted mistake {name} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(BANDIT_MUTANTS))
+def test_bandit_mutant_is_caught(name):
+    import bandit_pins as BP
+    with tempfile.TemporaryDirectory() as d:
+        lib = _build_mutant(name, d)
+        caught = []
+        for check in BP.ALL_BANDIT_CHECKS:
+            try:
+                with np.errstate(all="ignore"):
+                    check(lambda K, policy: oracle.Bandit(K, policy, lib=lib))
             except Exception as e:  # noqa: BLE001 - any failure counts as caught
                 caught.append((check.__name__, type(e).__name__))
                 break
