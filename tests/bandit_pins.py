@@ -106,7 +106,31 @@ def check_thompson_draw(make):
     th0 = 1 + math.sqrt(-2 * math.log(0.5)) * math.cos(math.pi) / math.sqrt(2)
     th1 = 0 + math.sqrt(-2 * math.log(1 - 0.999)) / math.sqrt(3)
     assert a == (0 if th0 > th1 else 1) and a == 1
+    # z0 = 0 (cos(pi/2)), z1 = sqrt(-2 ln 0.044) = 2.4993: theta = (1, 2.4993/sqrt 3
+    # = 1.443) -> arm 1; a posterior spread of 1/(N+1) instead of 1/sqrt(N+1) would
+    # give theta1 = 0.833 and pick arm 0
+    b = prepared()
+    assert b.step([0], 1, [0.5, 0.956], [0.25, 0.0]) == 1
+
+
+def check_thompson_choice_frequency(make):
+    """With N = (2, 1), R = (1, 0) the posterior draws are theta_k ~ Normal(R_k/N_k,
+    1/(N_k + 1)), so arm 1 is chosen with probability Phi((0 - 1/2) / sqrt(1/3 + 1/2))
+    = 0.292 (0.203 with a spread of 1/(N_k + 1)); over 20,000 draws (steps with an empty batch, which add no reward)
+    the frequency stays within 5 standard errors of it."""
+    b = make(2, THOMPSON)
+    for x in ([], [1], [0], [0]):
+        b.step(x, 1, [0, 0], [0, 0])
+    assert b.N.tolist() == [2.0, 1.0] and b.R.tolist() == [1.0, 0.0]
+    rng = np.random.default_rng(7)
+    n, hits = 20_000, 0
+    for _ in range(n):
+        hits += b.step([], 1, rng.random(2), rng.random(2)) == 1
+    p = 0.5 * math.erfc(0.5 / math.sqrt(1.0 / 3.0 + 0.5) / math.sqrt(2.0))
+    se = math.sqrt(p * (1 - p) / n)
+    assert abs(hits / n - p) < 5 * se, (hits / n, p)
 
 
 ALL_BANDIT_CHECKS = [check_reward_is_accepted_fraction, check_ucb1_hand_steps, check_ties_and_unrewarded_first,
-                     check_thompson_hand_steps, check_thompson_draw, check_regret_within_ucb1_bound]
+                     check_thompson_hand_steps, check_thompson_draw, check_thompson_choice_frequency,
+                     check_regret_within_ucb1_bound]
