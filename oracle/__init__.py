@@ -59,6 +59,8 @@ def load_library(path: str):
     lib.sv_oracle_bandit_step.argtypes = [p, ctypes.c_int, ctypes.c_int, p, p, p, p, ctypes.c_int, ctypes.c_int,
                                           p, p]
     lib.sv_oracle_bandit_step.restype = ctypes.c_int
+    lib.sv_oracle_bandit_simulate.argtypes = [p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, p, p, p]
+    lib.sv_oracle_bandit_simulate.restype = ctypes.c_int
     return lib
 
 
@@ -208,3 +210,20 @@ class Bandit:
         if rc != 0:
             raise ValueError("bad bandit arguments")
         return int(self.arm[0])
+
+
+def bandit_simulate(mu, T: int, policy: int, uniforms: np.ndarray, lib=None, with_state: bool = False):
+    """Regret of each run of the simulation (``sv_oracle_bandit_simulate``), and
+    with ``with_state`` each run's final [t, arm, N, R]."""
+    lib = _load() if lib is None else lib
+    mu = np.ascontiguousarray(mu, dtype=np.float64).reshape(-1)
+    K = mu.size
+    uniforms = np.ascontiguousarray(uniforms, dtype=np.float32)
+    runs = uniforms.shape[0]
+    assert uniforms.shape == (runs, T + 1, 2 * K + 1)
+    regret = np.empty(runs, np.float64)
+    state = np.empty((runs, 2 + 2 * K), np.float64)
+    if lib.sv_oracle_bandit_simulate(_ptr(mu), K, int(T), int(policy), runs, _ptr(uniforms), _ptr(regret),
+                                     _ptr(state)) != 0:
+        raise ValueError("bad bandit simulation arguments")
+    return (regret, state) if with_state else regret

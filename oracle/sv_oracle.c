@@ -530,3 +530,50 @@ int sv_oracle_bandit_step(const int32_t* n_accepted, int B, int gamma, double* t
     *arm = pick;
     return 0;
 }
+
+/*
+ * The regret simulation [FlashSpec, Resultados Principais, "Desempenho do
+ * Bandit": T rounds against K arms whose rewards are Bernoulli].  Each run
+ * composes sv_oracle_bandit_step with one sequence and gamma = 1, so a reward is
+ * 0 or 1 accepted drafts.  uniforms[run][s][2K+1], s in [0, T]: row s holds the
+ * step's u1 (K), u2 (K) and the round's reward draw r.  Step 0 (no reward yet)
+ * makes the first choice from row 0; round s = 1..T adds the gap mu_max -
+ * mu[arm] of the arm in play to the run's regret, then draws its reward
+ * (r_s < mu[arm]) and steps with row s.  out_regret[run]; out_state, if not
+ * null, gets each run's final [t, arm, N[K], R[K]].
+ */
+int sv_oracle_bandit_simulate(const double* mu, int K, int T, int policy, int runs, const float* uniforms,
+                              double* out_regret, double* out_state)
+{
+    if (K < 1 || K > 16 || T < 0 || runs < 0) return -1;
+    double mu_max = mu[0];
+    for (int k = 1; k < K; ++k)
+        if (mu[k] > mu_max) mu_max = mu[k];
+    const long long row = 2 * K + 1;
+    for (int r = 0; r < runs; ++r) {
+        const float* u = uniforms + (long long)r * (T + 1) * row;
+        double t = 0.0, N[16] = {0}, Rs[16] = {0}, regret = 0.0;
+        int32_t arm = -1;
+        sv_oracle_bandit_step(NULL, 0, 1, &t, &arm, N, Rs, K, policy, u, u + K);
+        for (int s = 1; s <= T; ++s) {
+            const float* us = u + (long long)s * row;
+            int32_t reward = 0;
+            if (arm >= 0) {
+                regret += mu_max - mu[arm];
+                reward = (double)us[2 * K] < mu[arm] ? 1 : 0;
+            }
+            sv_oracle_bandit_step(&reward, 1, 1, &t, &arm, N, Rs, K, policy, us, us + K);
+        }
+        out_regret[r] = regret;
+        if (out_state) {
+            double* o = out_state + (long long)r * (2 + 2 * K);
+            o[0] = t;
+            o[1] = (double)arm;
+            for (int k = 0; k < K; ++k) {
+                o[2 + k] = N[k];
+                o[2 + K + k] = Rs[k];
+            }
+        }
+    }
+    return 0;
+}

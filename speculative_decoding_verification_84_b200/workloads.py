@@ -258,3 +258,13 @@ def make_random(B: int, gamma: int, V: int, dtype: str, *, seed: int, T=1.0,
         toks[b] = gumbel_max_tokens(_stored_to_f64(dft[b], dtype), float(temp[b]), gu[b])
     return Workload(f"random_{B}x{gamma}x{V}_{dtype}", dtype, tgt, dft, toks, temp,
                     draw_uniforms(rng, (B, gamma)), draw_uniforms(rng, (B,)))
+
+
+def bandit_uniforms(runs: int, T: int, K: int, seed: int) -> np.ndarray:
+    """Uniforms of the draft-selection regret simulation: [runs][T + 1][2K + 1]
+    float32 in (0, 1), row s holding step s's u1 (K values) and u2 (K values),
+    then round s's reward draw.  Each run is seeded on its own (stream 7, key run)."""
+    out = np.empty((runs, T + 1, 2 * K + 1), np.float32)
+    for r in range(runs):
+        out[r] = draw_uniforms(_rng(seed, 7, r), (T + 1, 2 * K + 1))
+    return out

@@ -134,3 +134,67 @@ def check_thompson_choice_frequency(make):
 ALL_BANDIT_CHECKS = [check_reward_is_accepted_fraction, check_ucb1_hand_steps, check_ties_and_unrewarded_first,
                      check_thompson_hand_steps, check_thompson_draw, check_thompson_choice_frequency,
                      check_regret_within_ucb1_bound]
+
+
+# ---------------------------------------------------------------------------
+# The regret simulation (``oracle.bandit_simulate``).  Each check takes
+# ``sim(mu, T, policy, uniforms) -> (regret[runs], state[runs][2 + 2K])`` and the
+# bandit factory ``make(K, policy)`` of the same library.
+
+def _uniforms(runs, T, K, seed):
+    from speculative_decoding_verification_84_b200.workloads import bandit_uniforms
+    return bandit_uniforms(runs, T, K, seed)
+
+
+def check_sim_is_composed_steps(sim, make):
+    """Every run equals the loop written out with single steps: step 0 chooses from
+    row 0; round s adds the gap of the arm in play, rewards it with (r_s < mu) and
+    steps with row s."""
+    mu, T = (0.5, 0.7, 0.62), 300
+    K = len(mu)
+    for policy in (UCB1, THOMPSON):
+        U = _uniforms(3, T, K, 11 + policy)
+        regret, state = sim(mu, T, policy, U)
+        for r in range(U.shape[0]):
+            b = make(K, policy)
+            arm = b.step([], 1, U[r, 0, :K], U[r, 0, K:2 * K])
+            reg = 0.0
+            for s_ in range(1, T + 1):
+                reg += max(mu) - mu[arm]
+                rew = int(float(U[r, s_, 2 * K]) < mu[arm])
+                arm = b.step([rew], 1, U[r, s_, :K], U[r, s_, K:2 * K])
+            assert reg == regret[r], (policy, r, reg, regret[r])
+            want = [b.t[0], float(arm), *b.N.tolist(), *b.R.tolist()]
+            assert state[r].tolist() == want, (policy, r)
+
+
+def check_sim_degenerate(sim, make):
+    """One arm, or arms of equal means: no regret; every round is rewarded once."""
+    T = 200
+    regret, state = sim((0.4,), T, UCB1, _uniforms(2, T, 1, 3))
+    assert regret.tolist() == [0.0, 0.0] and state[:, 0].tolist() == [T, T] and state[:, 2].tolist() == [T, T]
+    for policy in (UCB1, THOMPSON):
+        regret, state = sim((0.5, 0.5), T, policy, _uniforms(2, T, 2, 4))
+        assert regret.tolist() == [0.0, 0.0] and (state[:, 2] + state[:, 3]).tolist() == [T, T]
+
+
+def check_sim_regret_bound(sim, make):
+    """Resultados Principais: T = 10,000, K = 3 (means (0.75, 0.6, 0.45), the pages'
+    are not given): mean UCB1 regret under Auer et al.'s bound, Thompson sampling
+    below UCB1, and every run's regret the sum of gap_k * N_k (N_k counts the
+    rounds arm k was played, each rewarded once)."""
+    mu, T, K = (0.75, 0.6, 0.45), 10_000, 3
+    gaps = [max(mu) - m for m in mu]
+    bound = sum(8 * math.log(T) / d for d in gaps if d > 0) + (1 + math.pi ** 2 / 3) * sum(gaps)
+    ru, su = sim(mu, T, UCB1, _uniforms(8, T, K, 21))
+    rt, st = sim(mu, T, THOMPSON, _uniforms(8, T, K, 22))
+    assert ru.mean() <= bound, (ru.mean(), bound)
+    assert rt.mean() < ru.mean(), (rt.mean(), ru.mean())
+    for regret, state in ((ru, su), (rt, st)):
+        for r in range(regret.size):
+            N = state[r, 2:2 + K]
+            assert N.sum() == T and state[r, 0] == T
+            assert abs(regret[r] - sum(g * n for g, n in zip(gaps, N))) < 1e-9 * T
+
+
+ALL_SIM_CHECKS = [check_sim_is_composed_steps, check_sim_degenerate, check_sim_regret_bound]

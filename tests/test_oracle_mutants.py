@@ -76,10 +76,21 @@ BANDIT_MUTANTS = {
     "bandit_reward_to_arm0": ("N[*arm] += 1.0;\n        R[*arm] += reward;", "N[*arm] += 1.0;\n        R[0] += reward;"),
 }
 
+BANDIT_SIM_MUTANTS = {
+    "sim_gap_from_first_arm": ("if (mu[k] > mu_max) mu_max = mu[k];", ";"),
+    "sim_reward_draw_of_last_row": ("reward = (double)us[2 * K] < mu[arm] ? 1 : 0;",
+                                    "reward = (double)us[-1] < mu[arm] ? 1 : 0;"),
+    "sim_reward_inverted": ("reward = (double)us[2 * K] < mu[arm] ? 1 : 0;",
+                            "reward = (double)us[2 * K] < mu[arm] ? 0 : 1;"),
+    "sim_u2_from_u1": ("sv_oracle_bandit_step(&reward, 1, 1, &t, &arm, N, Rs, K, policy, us, us + K);",
+                       "sv_oracle_bandit_step(&reward, 1, 1, &t, &arm, N, Rs, K, policy, us, us);"),
+    "sim_regret_after_step": ("regret += mu_max - mu[arm];", ";"),
+}
+
 
 def _build_mutant(name, tmpdir):
     src = open(SRC).read()
-    old, new = {**MUTANTS, **TOPF_MUTANTS, **BANDIT_MUTANTS}[name]
+    old, new = {**MUTANTS, **TOPF_MUTANTS, **BANDIT_MUTANTS, **BANDIT_SIM_MUTANTS}[name]
     assert src.count(old) == 1, f"mutation site for {name} not unique"
     path = os.path.join(tmpdir, f"{name}.c")
     with open(path, "w") as f:
@@ -158,6 +169,23 @@ def test_bandit_mutant_is_caught(name):
             try:
                 with np.errstate(all="ignore"):
                     check(lambda K, policy: oracle.Bandit(K, policy, lib=lib))
+            except Exception as e:  # noqa: BLE001 - any failure counts as caught
+                caught.append((check.__name__, type(e).__name__))
+                break
+        assert caught, f"planted mistake {name} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(BANDIT_SIM_MUTANTS))
+def test_bandit_sim_mutant_is_caught(name):
+    import bandit_pins as BP
+    with tempfile.TemporaryDirectory() as d:
+        lib = _build_mutant(name, d)
+        clean = oracle.load_library(oracle.build())
+        caught = []
+        for check in BP.ALL_SIM_CHECKS:
+            try:
+                check(lambda mu, T, policy, U: oracle.bandit_simulate(mu, T, policy, U, lib=lib, with_state=True),
+                      lambda K, policy: oracle.Bandit(K, policy, lib=clean))
             except Exception as e:  # noqa: BLE001 - any failure counts as caught
                 caught.append((check.__name__, type(e).__name__))
                 break
