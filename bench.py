@@ -322,6 +322,112 @@ def config_line(c, peak, peak_kind, hot=False, budget_ms=20.0):
     }
 
 
+def graph_ms(stream, fn, k, n_copies):
+    """Mean ms per call of fn(0), fn(1), ... replayed from a CUDA graph of one round
+    over the input copies (at least 16 calls), at least k calls timed between two
+    events on the launching stream."""
+    import torch
+    n = n_copies * max(1, -(-16 // n_copies))
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fn(i)
+    reps = max(3, -(-k // n))
+    with torch.cuda.stream(stream):  # replay() launches on the current stream
+        g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / (reps * n)
+
+
+# arms of the regret simulation: the pages give T = 10,000 rounds and K = 3 arms
+# but not the means; these give Auer et al.'s UCB1 bound 518.8 (the pages: ~526)
+BANDIT_MU = (0.8, 0.6, 0.3)
+BANDIT_T = 10_000
+BANDIT_RUNS = 1024
+
+
+def bandit_row_line(w, dev, lib, binding, cpu_seconds=2.0):
+    """Draft selection on the device.  (1) spec_verify_bandit_step right after
+    spec_verify on workload w, its reward summed from that call's n_accepted on
+    the device: the bandit step alone and the time it adds to a verification,
+    both as CUDA graph replays over the input copies.  (2) The regret simulation
+    at the pages' size (T = 10,000 rounds, K = 3 Bernoulli arms) over
+    BANDIT_RUNS independent runs per policy, one launch each, with the mean regret
+    beside Auer et al.'s UCB1 bound; the fp64 oracle runs a sample of the same
+    runs on the host cores for comparison."""
+    import math
+    import torch
+    from speculative_decoding_verification_84_b200 import workloads as W
+    import oracle
+    c = Caller(w, dev, lib, binding)
+    K = 3
+    rng = np.random.default_rng(3)
+    u1 = torch.from_numpy(W.draw_uniforms(rng, (K,))).to(dev)
+    u2 = torch.from_numpy(W.draw_uniforms(rng, (K,))).to(dev)
+    out = {"workload": w.name, "K": K}
+    for policy, pname in ((binding.BANDIT_UCB1, "ucb1"), (binding.BANDIT_THOMPSON, "thompson")):
+        state = binding.bandit_state(K, dev, stream=c.stream)
+        arm = torch.empty(1, dtype=torch.int32, device=dev)
+
+        def step(i):
+            binding.bandit_step(c.out_n, c.gamma, state, policy, u1, u2, arm, stream=c.stream)
+
+        def both(i):
+            c.call(i)
+            step(i)
+
+        with torch.cuda.stream(c.stream):
+            for i in range(4):
+                both(i)
+        ms_v = graph_ms(c.stream, c.call, 200, c.n_copies)
+        ms_vb = graph_ms(c.stream, both, 200, c.n_copies)
+        ms_b = graph_ms(c.stream, step, 2000, c.n_copies)
+        out[f"us_per_step_{pname}"] = 1e3 * ms_b
+        out[f"us_added_to_verify_{pname}"] = 1e3 * (ms_vb - ms_v)
+    out["us_per_verify_call"] = 1e3 * ms_v
+    del c
+    torch.cuda.empty_cache()
+
+    mu = BANDIT_MU
+    gaps = [max(mu) - m for m in mu]
+    bound = sum(8 * math.log(BANDIT_T) / d for d in gaps if d > 0) + (1 + math.pi ** 2 / 3) * sum(gaps)
+    U = W.bandit_uniforms(BANDIT_RUNS, BANDIT_T, K, seed=2002)
+    Ud = torch.from_numpy(U).to(dev)
+    mud = torch.tensor(mu, dtype=torch.float64, device=dev)
+    sim = {"mu": list(mu), "T": BANDIT_T, "runs": BANDIT_RUNS, "ucb1_bound": bound,
+           "pages": {"ucb1_regret": 100.2, "ucb1_bound": 526, "thompson_regret": 18.9}}
+    for policy, pname in ((binding.BANDIT_UCB1, "ucb1"), (binding.BANDIT_THOMPSON, "thompson")):
+        binding.bandit_simulate(mud, BANDIT_T, policy, Ud)  # warm
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        reg = binding.bandit_simulate(mud, BANDIT_T, policy, Ud)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        r = reg.cpu().numpy()
+        # the oracle on a sample of the same runs, for comparison
+        n_cpu, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < cpu_seconds / 2 and n_cpu < BANDIT_RUNS:
+            oracle.bandit_simulate(mu, BANDIT_T, policy, U[n_cpu:n_cpu + 8])
+            n_cpu += 8
+        cpu_s = time.perf_counter() - t0
+        sim[pname] = {"regret_mean": float(r.mean()), "regret_sd": float(r.std()), "ms": ms,
+                      "steps_per_s": BANDIT_RUNS * BANDIT_T / (ms / 1e3),
+                      "cpu_baseline": {"kind": "oracle", "cores": 1, "steps_per_s": n_cpu * BANDIT_T / cpu_s,
+                                       "sample": f"{n_cpu} of the runs, {cpu_s:.2f} s"}}
+    out["simulation"] = sim
+    return out
+
+
 def cache_row_line(w, dev, lib, binding, peak, peak_kind, budget_ms=20.0):
     """The speculation-cache row on one workload: spec_verify_topf with the
     geometric fan-out of a 64-slot budget at acceptance rate 0.7 (then at most 32
@@ -366,24 +472,7 @@ def cache_row_line(w, dev, lib, binding, peak, peak_kind, budget_ms=20.0):
             raise RuntimeError(binding.status_string(rc))
 
     def graph_time(fn, k):
-        n = c.n_copies * max(1, -(-16 // c.n_copies))
-        g = torch.cuda.CUDAGraph()
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=c.stream):
-            for i in range(n):
-                fn(i)
-        reps = max(3, -(-k // n))
-        with torch.cuda.stream(c.stream):
-            g.replay()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(c.stream)
-        with torch.cuda.stream(c.stream):
-            for _ in range(reps):
-                g.replay()
-        e1.record(c.stream)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / (reps * n)
+        return graph_ms(c.stream, fn, k, c.n_copies)
 
     with torch.cuda.stream(c.stream):
         for i in range(4):
@@ -523,6 +612,8 @@ def run_ours(args):
             del wc
             torch.cuda.empty_cache()
         per_config["cache_row_c3"] = cache_row_line(W.make_workload(WORKLOAD), dev, lib, binding, peak, peak_kind)
+        torch.cuda.empty_cache()
+        per_config["bandit_row_c3"] = bandit_row_line(W.make_workload(WORKLOAD), dev, lib, binding)
         torch.cuda.empty_cache()
 
     cpu = None

@@ -253,6 +253,82 @@ sv_status spec_verify_cache_lookup(const int32_t* out_tokens, const int32_t* out
                                    const int32_t* cache_tokens, const int32_t* fanout, int B, int gamma,
                                    int32_t* out_slot, struct CUstream_st* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Draft selection as a K-armed bandit, on the device [FlashSpec, Metodologia 2,
+ * "Selecao de Rascunho via Bandit Online": each decoding step picks one of K
+ * draft models (arms) from past acceptances only; the reward is the fraction of
+ * draft tokens accepted; UCB1 and Thompson sampling.  Resultados Principais,
+ * "Desempenho do Bandit": regret over T rounds].  The reward is summed from
+ * spec_verify's out_n_accepted on the device, so no per-sequence count crosses
+ * to the host; the chosen arm is one int32 in device memory.
+ *
+ * State (caller-owned device doubles, spec_verify_bandit_state_size(K) bytes):
+ *   [0] t = rewards seen, [1] the arm chosen last (-1: none yet),
+ *   [2, 2+K) N_k = rewards seen for arm k, [2+K, 2+2K) R_k = their sum.
+ * The state is the only memory a bandit keeps; steps on one state must be
+ * ordered (same stream, or events).
+ */
+#define SV_MAX_ARMS 16
+#define SV_BANDIT_UCB1 0
+#define SV_BANDIT_THOMPSON 1
+
+/* Bytes of one bandit's state, 8 * (2 + 2K); 0 for K outside [1, SV_MAX_ARMS]. */
+size_t spec_verify_bandit_state_size(int K);
+
+/* Enqueue writing the empty state (t = 0, arm = -1, N = R = 0) to `state`
+ * (device, 8-byte aligned). */
+sv_status spec_verify_bandit_init(double* state, int K, struct CUstream_st* stream);
+
+/*
+ * One decoding step of the bandit:
+ *  (1) if an arm in [0, K) was chosen last and B > 0, it earns the reward
+ *      sum_b n_accepted[b] / (B * gamma) (the batch's accepted fraction, summed
+ *      exactly in 64-bit integers, divided in fp64): N_arm += 1, R_arm += reward,
+ *      t += 1;
+ *  (2) the next arm: the smallest arm never rewarded (N_k = 0) if any; else the
+ *      largest score, the smaller k on ties, where
+ *        SV_BANDIT_UCB1 (Auer, Cesa-Bianchi and Fischer, 2002):
+ *            R_k/N_k + sqrt(2 ln t / N_k)
+ *        SV_BANDIT_THOMPSON, Gaussian posteriors (Agrawal and Goyal, 2013):
+ *            R_k/N_k + z_k / sqrt(N_k + 1),
+ *            z_k = sqrt(-2 ln(1 - u1[k])) cos(2 pi u2[k])   (Box-Muller);
+ *      a score that is NaN or -inf never wins; when none wins the arm is -1 and
+ *      the next step rewards nothing.
+ *  (3) state[1] and *out_arm (if not null) = that arm.
+ *
+ *   n_accepted  [B] int32 (spec_verify's out_n_accepted); B = 0 rewards nothing
+ *   u1, u2      [K] float in [0, 1), this step's uniforms; read for Thompson
+ *               sampling only (may be null for UCB1)
+ *   state       as above;  out_arm  optional [1] int32
+ * All pointers are device memory.  The kernel waits (programmatic dependent
+ * launch) for the work before it on the stream, so it can follow spec_verify
+ * directly.  Returns SV_ERR_INVALID_ARG for K outside [1, SV_MAX_ARMS], B < 0,
+ * gamma < 1, an unknown policy or a missing pointer, before any launch.
+ * Scores are fp64 (log, cos, sqrt of the CUDA math library): compared with an
+ * exact evaluation a choice can differ only between arms whose scores agree to
+ * within a few units in the last place.  The unrewarded-first rule and the
+ * Gaussian form of the Thompson posterior are this library's readings.
+ */
+sv_status spec_verify_bandit_step(const int32_t* n_accepted, int B, int gamma, int policy,
+                                  const float* u1, const float* u2, double* state, int K,
+                                  int32_t* out_arm, struct CUstream_st* stream);
+
+/*
+ * The regret simulation: `runs` independent bandits, each played for T rounds
+ * against K Bernoulli arms of means mu[k], with one sequence and gamma = 1 per
+ * step (a reward is 0 or 1).  uniforms [runs][T+1][2K+1] float: row s holds
+ * step s's u1 (K values), u2 (K values), then round s's reward draw r_s.  Step 0
+ * (nothing to reward) chooses from row 0; round s = 1..T adds the gap
+ * max_k mu_k - mu[arm] of the arm in play to the run's regret, rewards that arm
+ * with (r_s < mu[arm]) and steps with row s.
+ *   out_regret [runs] double;  out_state optional [runs][2+2K] double: each
+ *   run's final state.  mu [K] double.  All device pointers.
+ */
+sv_status spec_verify_bandit_simulate(const double* mu, int K, int T, int policy, int runs,
+                                      const float* uniforms, double* out_regret, double* out_state,
+                                      struct CUstream_st* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,8 +21,12 @@ SV_DTYPE_F32, SV_DTYPE_BF16 = 0, 1
 ROW_BAD_TOKEN, ROW_BAD_LOGITS, ROW_BAD_TEMPERATURE, ROW_RESIDUAL_ZERO, ROW_BAD_UNIFORM = 1, 2, 4, 8, 16
 EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_init",
             "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc",
-            "spec_verify_fanout", "spec_verify_topf", "spec_verify_cache_lookup")
+            "spec_verify_fanout", "spec_verify_topf", "spec_verify_cache_lookup",
+            "spec_verify_bandit_state_size", "spec_verify_bandit_init", "spec_verify_bandit_step",
+            "spec_verify_bandit_simulate")
 MAX_TOPF = 32
+MAX_ARMS = 16
+BANDIT_UCB1, BANDIT_THOMPSON = 0, 1
 
 _lib = None
 
@@ -60,6 +64,14 @@ def load_library(path: str = LIB_PATH):
     lib.spec_verify_topf.restype = i32
     lib.spec_verify_cache_lookup.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp]
     lib.spec_verify_cache_lookup.restype = i32
+    lib.spec_verify_bandit_state_size.argtypes = [i32]
+    lib.spec_verify_bandit_state_size.restype = sz
+    lib.spec_verify_bandit_init.argtypes = [vp, i32, vp]
+    lib.spec_verify_bandit_init.restype = i32
+    lib.spec_verify_bandit_step.argtypes = [vp, i32, i32, i32, vp, vp, vp, i32, vp, vp]
+    lib.spec_verify_bandit_step.restype = i32
+    lib.spec_verify_bandit_simulate.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+    lib.spec_verify_bandit_simulate.restype = i32
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -235,6 +247,72 @@ def cache_lookup(out_tokens: torch.Tensor, n_accepted: torch.Tensor, cache_token
     if st != SV_OK:
         raise SpecVerifyError(st, status_string(st))
     return slot
+
+
+def _raise_if(st: int):
+    if st != SV_OK:
+        raise SpecVerifyError(st, status_string(st))
+
+
+def bandit_state(K: int, device="cuda", stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """A new bandit state on ``device`` ([2 + 2K] float64: t, arm, N, R), set to
+    the empty state by the library on ``stream``."""
+    lib = load_library()
+    nbytes = lib.spec_verify_bandit_state_size(int(K))
+    if nbytes == 0:
+        raise SpecVerifyError(1, f"K must be in [1, {MAX_ARMS}]")
+    device = torch.device(device)
+    state = torch.empty((nbytes // 8,), dtype=torch.float64, device=device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_bandit_init(state.data_ptr(), int(K), s.cuda_stream))
+    return state
+
+
+def bandit_step(n_accepted: torch.Tensor, gamma: int, state: torch.Tensor, policy: int = BANDIT_UCB1,
+                u1: torch.Tensor | None = None, u2: torch.Tensor | None = None,
+                out_arm: torch.Tensor | None = None, *, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Reward the arm chosen last with the batch's accepted fraction and choose the
+    next arm, on the device; returns ``out_arm`` ([1] int32, device)."""
+    lib = load_library()
+    device = state.device
+    K = (state.numel() - 2) // 2
+    _check(state, "state", torch.float64, (2 + 2 * K,), device)
+    B = n_accepted.numel()
+    _check(n_accepted, "n_accepted", torch.int32, (B,), device)
+    for name, u in (("u1", u1), ("u2", u2)):
+        if u is not None:
+            _check(u, name, torch.float32, (K,), device)
+    if out_arm is None:
+        out_arm = torch.empty((1,), dtype=torch.int32, device=device)
+    _check(out_arm, "out_arm", torch.int32, (1,), device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_bandit_step(n_accepted.data_ptr(), B, int(gamma), int(policy),
+                                              u1.data_ptr() if u1 is not None else None,
+                                              u2.data_ptr() if u2 is not None else None,
+                                              state.data_ptr(), K, out_arm.data_ptr(), s.cuda_stream))
+    return out_arm
+
+
+def bandit_simulate(mu: torch.Tensor, T: int, policy: int, uniforms: torch.Tensor, *, with_state: bool = False,
+                    stream: torch.cuda.Stream | None = None):
+    """Regret of each run of the simulation ([runs] float64, device); with
+    ``with_state`` also each run's final state ([runs][2 + 2K])."""
+    lib = load_library()
+    device = mu.device
+    K = mu.numel()
+    _check(mu, "mu", torch.float64, (K,), device)
+    runs = uniforms.shape[0] if uniforms.dim() == 3 else -1
+    _check(uniforms, "uniforms", torch.float32, (runs, int(T) + 1, 2 * K + 1), device)
+    regret = torch.empty((runs,), dtype=torch.float64, device=device)
+    state = torch.empty((runs, 2 + 2 * K), dtype=torch.float64, device=device) if with_state else None
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_bandit_simulate(mu.data_ptr(), K, int(T), int(policy), runs, uniforms.data_ptr(),
+                                                  regret.data_ptr(), state.data_ptr() if with_state else None,
+                                                  s.cuda_stream))
+    return (regret, state) if with_state else regret
 
 
 def to_device(w, device="cuda"):

@@ -30,6 +30,7 @@
 #include "sv_pass.cuh"
 #include "sv_small.cuh"
 #include "sv_topf.cuh"
+#include "sv_bandit.cuh"
 
 namespace {
 
@@ -622,5 +623,61 @@ extern "C" sv_status spec_verify_cache_lookup(const int32_t* out_tokens, const i
     const unsigned grid = (unsigned)cdiv(B, 256);
     sv::sv_cache_lookup<<<grid, 256, 0, (cudaStream_t)stream>>>(out_tokens, out_n_accepted, cache_tokens, g,
                                                                   out_slot);
+    return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+static_assert(sv::kBanditMaxArms == SV_MAX_ARMS, "arm limit");
+
+extern "C" size_t spec_verify_bandit_state_size(int K)
+{
+    return (K < 1 || K > SV_MAX_ARMS) ? 0 : sizeof(double) * (size_t)(2 + 2 * K);
+}
+
+extern "C" sv_status spec_verify_bandit_init(double* state, int K, struct CUstream_st* stream)
+{
+    if (!state || K < 1 || K > SV_MAX_ARMS) return SV_ERR_INVALID_ARG;
+    if (!aligned(state, 8)) return SV_ERR_MISALIGNED;
+    sv::sv_bandit_init<<<1, 64, 0, (cudaStream_t)stream>>>(state, K);
+    return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+extern "C" sv_status spec_verify_bandit_step(const int32_t* n_accepted, int B, int gamma, int policy,
+                                             const float* u1, const float* u2, double* state, int K,
+                                             int32_t* out_arm, struct CUstream_st* stream)
+{
+    if (B < 0 || gamma < 1 || K < 1 || K > SV_MAX_ARMS || !state || (B > 0 && !n_accepted) ||
+        (policy != SV_BANDIT_UCB1 && policy != SV_BANDIT_THOMPSON) ||
+        (policy == SV_BANDIT_THOMPSON && (!u1 || !u2)))
+        return SV_ERR_INVALID_ARG;
+    if (!aligned(n_accepted, 4) || !aligned(u1, 4) || !aligned(u2, 4) || !aligned(state, 8) || !aligned(out_arm, 4))
+        return SV_ERR_MISALIGNED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(sv::kBanditStepThreads);
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e =
+        cudaLaunchKernelEx(&cfg, sv::sv_bandit_step, n_accepted, B, gamma, policy, u1, u2, state, K, out_arm);
+    return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+extern "C" sv_status spec_verify_bandit_simulate(const double* mu, int K, int T, int policy, int runs,
+                                                 const float* uniforms, double* out_regret, double* out_state,
+                                                 struct CUstream_st* stream)
+{
+    if (!mu || K < 1 || K > SV_MAX_ARMS || T < 0 || runs < 0 ||
+        (policy != SV_BANDIT_UCB1 && policy != SV_BANDIT_THOMPSON) || (runs > 0 && (!uniforms || !out_regret)))
+        return SV_ERR_INVALID_ARG;
+    if (!aligned(mu, 8) || !aligned(uniforms, 4) || !aligned(out_regret, 8) || !aligned(out_state, 8))
+        return SV_ERR_MISALIGNED;
+    if (runs == 0) return SV_OK;
+    constexpr int kRunsPerCta = sv::kBanditSimThreads / 32;
+    const unsigned grid = (unsigned)cdiv(runs, kRunsPerCta);
+    sv::sv_bandit_simulate<<<grid, sv::kBanditSimThreads, 0, (cudaStream_t)stream>>>(mu, K, T, policy, runs, uniforms,
+                                                                                       out_regret, out_state);
     return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }

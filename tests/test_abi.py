@@ -101,3 +101,35 @@ def test_fanout_host_matches_oracle(lib):
     assert lib.spec_verify_fanout(1.5, 2, 4, F.ctypes.data) != 0
     assert lib.spec_verify_fanout(0.5, 0, 4, F.ctypes.data) != 0
     assert lib.spec_verify_fanout(0.5, 2, -1, F.ctypes.data) != 0
+
+
+def test_bandit_host_validation(lib):
+    """State size and the bandit entry points' host checks (no launch)."""
+    vp = ctypes.c_void_p
+    good = vp(1 << 20)
+    assert lib.spec_verify_bandit_state_size(3) == 8 * 8
+    assert lib.spec_verify_bandit_state_size(16) == 8 * 34
+    assert lib.spec_verify_bandit_state_size(0) == 0 and lib.spec_verify_bandit_state_size(17) == 0
+    assert lib.spec_verify_bandit_init(None, 3, None) == 1
+    assert lib.spec_verify_bandit_init(good, 17, None) == 1
+    assert lib.spec_verify_bandit_init(vp((1 << 20) + 4), 3, None) == 3
+    step = [good, 4, 5, 0, None, None, good, 3, None, None]
+    bad = list(step); bad[3] = 2                 # unknown policy
+    assert lib.spec_verify_bandit_step(*bad) == 1
+    bad = list(step); bad[3] = 1                 # Thompson sampling without uniforms
+    assert lib.spec_verify_bandit_step(*bad) == 1
+    bad = list(step); bad[2] = 0                 # gamma
+    assert lib.spec_verify_bandit_step(*bad) == 1
+    bad = list(step); bad[0] = None              # B > 0 without n_accepted
+    assert lib.spec_verify_bandit_step(*bad) == 1
+    bad = list(step); bad[6] = vp((1 << 20) + 4)  # state not 8-byte aligned
+    assert lib.spec_verify_bandit_step(*bad) == 3
+    sim = [good, 3, 100, 0, 4, good, good, None, None]
+    bad = list(sim); bad[1] = 0
+    assert lib.spec_verify_bandit_simulate(*bad) == 1
+    bad = list(sim); bad[2] = -1
+    assert lib.spec_verify_bandit_simulate(*bad) == 1
+    bad = list(sim); bad[5] = None
+    assert lib.spec_verify_bandit_simulate(*bad) == 1
+    zero = list(sim); zero[4] = 0                # no runs: nothing to launch
+    assert lib.spec_verify_bandit_simulate(*zero) == 0
