@@ -22,7 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "sv_oracle.c")
 _LIB = os.path.join(_HERE, "libsvoracle.so")
 
-ST_TOKEN, ST_ROW, ST_TEMP, ST_RESID0, ST_UNIFORM = 1, 2, 4, 8, 16
+ST_TOKEN, ST_ROW, ST_TEMP, ST_RESID0, ST_UNIFORM, ST_TREE = 1, 2, 4, 8, 16, 32
 RESIDUAL_MIN = 2.0 ** -18   # residual mass below this counts as vanished
 NEAR_ACCEPT, NEAR_CDF = 1, 2
 
@@ -61,6 +61,12 @@ def load_library(path: str):
     lib.sv_oracle_bandit_step.restype = ctypes.c_int
     lib.sv_oracle_bandit_simulate.argtypes = [p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, p, p, p]
     lib.sv_oracle_bandit_simulate.restype = ctypes.c_int
+    lib.sv_oracle_tree_verify.argtypes = [p, p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, p, p, p, p, p, p, p, p, ctypes.c_int]
+    lib.sv_oracle_tree_verify.restype = ctypes.c_int
+    lib.sv_oracle_tree_prune.argtypes = [p, ctypes.c_int, p, p, p, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, p, p]
+    lib.sv_oracle_tree_prune.restype = ctypes.c_int
     return lib
 
 
@@ -227,3 +233,64 @@ def bandit_simulate(mu, T: int, policy: int, uniforms: np.ndarray, lib=None, wit
                                      _ptr(state)) != 0:
         raise ValueError("bad bandit simulation arguments")
     return (regret, state) if with_state else regret
+
+
+@dataclasses.dataclass
+class TreeResult:
+    out_nodes: np.ndarray    # [B, N] int32: accepted nodes in path order, then -1
+    out_tokens: np.ndarray   # [B, N] int32: their tokens, the extra token, then -1
+    n_accepted: np.ndarray   # [B] int32
+    log_norm: np.ndarray     # [B, 2N] float64: target rows, then draft rows (NaN: not read)
+    row_status: np.ndarray   # [B] int32
+    near_tie: np.ndarray     # [B] int32 (1 accept test, 2 inverse CDF / fallback threshold)
+    accept_gap: np.ndarray   # [B] float64
+    cdf_gap: np.ndarray      # [B] float64
+
+
+def tree_verify(target, draft, parent, tokens, temperature, u_accept, u_resample, keep=None, *,
+                bf16: bool | None = None, n_threads: int = 0, lib=None) -> TreeResult:
+    """Tree verification (``sv_oracle_tree_verify``): target, draft [B, N, V];
+    parent, tokens, u_accept [B, N]; keep [B, N] or None."""
+    lib = _load() if lib is None else lib
+    target = np.ascontiguousarray(target)
+    draft = np.ascontiguousarray(draft)
+    if bf16 is None:
+        bf16 = target.dtype == np.uint16
+    B, N, V = target.shape
+    assert draft.shape == (B, N, V)
+    par = np.ascontiguousarray(parent, dtype=np.int32).reshape(B, N)
+    tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, N)
+    kp = None if keep is None else np.ascontiguousarray(keep, dtype=np.int32).reshape(B, N)
+    T = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    ua = np.ascontiguousarray(u_accept, dtype=np.float32).reshape(B, N)
+    ur = np.ascontiguousarray(u_resample, dtype=np.float32).reshape(B)
+    r = TreeResult(np.empty((B, N), np.int32), np.empty((B, N), np.int32), np.empty(B, np.int32),
+                   np.empty((B, 2 * N), np.float64), np.empty(B, np.int32), np.empty(B, np.int32),
+                   np.empty(B, np.float64), np.empty(B, np.float64))
+    rc = lib.sv_oracle_tree_verify(_ptr(target), _ptr(draft), int(bool(bf16)), _ptr(par), _ptr(tok),
+                                   None if kp is None else _ptr(kp), _ptr(T), _ptr(ua), _ptr(ur), B, N, V,
+                                   _ptr(r.out_nodes), _ptr(r.out_tokens), _ptr(r.n_accepted), _ptr(r.log_norm),
+                                   _ptr(r.row_status), _ptr(r.near_tie), _ptr(r.accept_gap), _ptr(r.cdf_gap),
+                                   int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"sv_oracle_tree_verify failed ({rc})")
+    return r
+
+
+def tree_prune(draft, parent, tokens, temperature, threshold: float, *, bf16: bool | None = None, lib=None):
+    """Cumulative draft log-probability of every node and the nodes kept at
+    ``threshold`` (``sv_oracle_tree_prune``): (keep [B, N] int32, cum [B, N])."""
+    lib = _load() if lib is None else lib
+    draft = np.ascontiguousarray(draft)
+    if bf16 is None:
+        bf16 = draft.dtype == np.uint16
+    B, N, V = draft.shape
+    par = np.ascontiguousarray(parent, dtype=np.int32).reshape(B, N)
+    tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, N)
+    T = np.ascontiguousarray(temperature, dtype=np.float32).reshape(B)
+    keep = np.empty((B, N), np.int32)
+    cum = np.empty((B, N), np.float64)
+    if lib.sv_oracle_tree_prune(_ptr(draft), int(bool(bf16)), _ptr(par), _ptr(tok), _ptr(T), float(threshold),
+                                B, N, V, _ptr(keep), _ptr(cum)) != 0:
+        raise ValueError("bad tree shape")
+    return keep, cum

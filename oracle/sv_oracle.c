@@ -577,3 +577,282 @@ int sv_oracle_bandit_simulate(const double* mu, int K, int T, int policy, int ru
     }
     return 0;
 }
+
+/*
+ * Tree verification [SpecLA, Metodologia 1, "Kernels de Verificacao de Topologia
+ * Conscientes": drafts shaped as chains or as branching trees; Speculative
+ * Speculative Decoding, "Significado e Impacto": compatible with token trees].
+ * The pages give no acceptance rule for several candidates; this follows the
+ * multi-candidate form of the same speculative-sampling rule (the form whose
+ * output law equals the target's when the children of a node are independent
+ * draws from q at that node):
+ *
+ *   At node c (first the root), P starts as the target's p at c.  The children of
+ *   c are tested in increasing index: child x is accepted iff
+ *       log u_x < log P(tok_x) - log q(tok_x),
+ *   q the draft's distribution at c.  After a rejection P becomes
+ *   norm(max(0, P - q)) -- or stays P when that mass is below 2^-18 (status bit 8,
+ *   the rule of sv_oracle_verify) -- and the next child is tested.  An accepted
+ *   child becomes c.  When no child of c is accepted, or c has none, the extra
+ *   token is drawn from P by the inverse CDF with u_resample, and the walk ends.
+ *   T == 0 (greedy): the first child whose token is the first argmax of target
+ *   row c is accepted; otherwise that argmax is the extra token.
+ *
+ * A chain (node i's parent i - 1) gives exactly sv_oracle_verify's result.
+ *
+ * Layout, sequence b with N nodes: node 0 is the root (the context verified so
+ * far); node i >= 1 carries the draft token tok[i] and its parent par[i] in
+ * [0, i); par[0] = -1.  target [B][N][V]: the target's next-token logits at node
+ * i's context (the path to i, tok[i] included); draft [B][N][V]: the draft's,
+ * the distribution node i's children were drawn from.  keep [B][N], optional:
+ * node i >= 1 takes part iff keep[i] != 0 and its parent takes part.
+ * u_accept [B][N]: the uniform of node i's test (entry 0 unused).
+ *
+ * P is held as weights w with P = w / S_w: w = p and S_w = 1 at first, then w =
+ * max(0, P - q) and S_w = its sum, so the first residual and its draw are
+ * sv_oracle_verify's bit for bit.
+ *
+ * Status: 4 bad temperature; 32 a parent index out of range; 1 a token of a
+ * node that takes part outside [0, V); 16 (T > 0) u_accept of a node that takes
+ * part, or u_resample, outside [0, 1) or NaN; 2 a row the walk reads (target row
+ * of every node visited; T > 0: the draft row of every visited node that has
+ * children taking part) is bad.  With 1, 2, 4, 16 or 32 nothing is emitted.
+ * Near ties: bit 1 at a test with |log u - delta| below 1e-6 (the first child
+ * of a node) or below 1e-6 + the relative error bound of P(tok) (later
+ * children: fp32 weights carry about 4e-6 relative error per rounding, tracked
+ * through the residual levels); bit 2 at a draw whose inverse-CDF gap is below
+ * 1e-6, plus the tracked error of the weights after two or more rejections, or
+ * whose residual mass lies within that of the 2^-18 threshold.
+ */
+#define ST_TREE 32
+#define ORACLE_EPS_W 4e-6
+
+static int tree_child_after(const int32_t* par, const int* in, int N, int c, int from)
+{
+    for (int i = from; i < N; ++i)
+        if (in[i] && par[i] == c) return i;
+    return -1;
+}
+
+static void tree_one(const void* tgt, const void* dft, int is_bf16, const int32_t* par, const int32_t* tok,
+                     const int32_t* keep, double T, const float* u_acc, double u_res, int N, int V, size_t b,
+                     int32_t* out_nodes, int32_t* out_tok, int32_t* out_n, double* lnorm, int32_t* status,
+                     int32_t* near, double* agap, double* cgap, double* wbuf, double* ebuf)
+{
+    int st = 0, nr = 0, in[64];
+    *agap = INFINITY;
+    *cgap = INFINITY;
+    for (int i = 0; i < N; ++i) { out_nodes[i] = -1; out_tok[i] = -1; }
+    for (int r = 0; r < 2 * N; ++r) lnorm[r] = NAN;
+    *out_n = 0;
+    *near = 0;
+    if (!(T == 0.0 || (isfinite(T) && T >= ORACLE_T_MIN))) { *status = ST_TEMP; return; }
+    if (par[0] != -1) st |= ST_TREE;
+    in[0] = 1;
+    for (int i = 1; i < N; ++i) {
+        if (par[i] < 0 || par[i] >= i) { st |= ST_TREE; in[i] = 0; continue; }
+        in[i] = in[par[i]] && (keep == NULL || keep[i] != 0);
+    }
+    for (int i = 1; i < N; ++i)
+        if (in[i] && (tok[i] < 0 || tok[i] >= V)) st |= ST_TOKEN;
+    if (T > 0.0) {
+        for (int i = 1; i < N; ++i)
+            if (in[i] && !(u_acc[i] >= 0.0f && u_acc[i] < 1.0f)) st |= ST_UNIFORM;
+        if (!(u_res >= 0.0 && u_res < 1.0)) st |= ST_UNIFORM;
+    }
+    if (st) { *status = st; return; }
+
+    const size_t base = b * (size_t)N * (size_t)V;
+    int c = 0, n = 0, k = -1;
+    if (T == 0.0) {
+        for (;;) {
+            const int a = row_argmax(tgt, is_bf16, base + (size_t)c * V, V);
+            if (a < 0) { st |= ST_ROW; break; }
+            int next = -1;
+            for (int i = tree_child_after(par, in, N, c, c + 1); i >= 0; i = tree_child_after(par, in, N, c, i + 1))
+                if (tok[i] == a) { next = i; break; }
+            if (next < 0) { k = a; break; }
+            out_nodes[n] = next;
+            ++n;
+            c = next;
+        }
+    } else {
+        for (;;) {
+            double lse_t, lse_d = 0.0;
+            const size_t trow = base + (size_t)c * V;
+            if (!row_lse(tgt, is_bf16, trow, V, T, &lse_t)) { st |= ST_ROW; break; }
+            lnorm[c] = lse_t;
+            const int first = tree_child_after(par, in, N, c, c + 1);
+            if (first >= 0) {
+                if (!row_lse(dft, is_bf16, trow, V, T, &lse_d)) { st |= ST_ROW; break; }
+                lnorm[N + c] = lse_d;
+            }
+            /* P = w / Sw, first the target's p at c */
+            double Sw = 1.0;
+            int level = 0;
+            for (int v = 0; v < V; ++v) {
+                wbuf[v] = exp(widen(tgt, is_bf16, trow + (size_t)v) / T - lse_t);
+                ebuf[v] = ORACLE_EPS_W * wbuf[v];
+            }
+            int next = -1;
+            double resid_gap = INFINITY;
+            for (int i = first; i >= 0; i = tree_child_after(par, in, N, c, i + 1)) {
+                const int x = tok[i];
+                const double lq = widen(dft, is_bf16, trow + (size_t)x) / T - lse_d;
+                const double lp = level == 0 ? widen(tgt, is_bf16, trow + (size_t)x) / T - lse_t
+                                             : log(wbuf[x]) - log(Sw);
+                const double delta = lp - lq;
+                const double lu = log((double)u_acc[i]);
+                /* a weight of exactly 0 rejects whatever u is: no band */
+                const double band = level == 0 ? ORACLE_NEAR
+                                    : (wbuf[x] > 0.0 ? ORACLE_NEAR + ebuf[x] / wbuf[x] + ORACLE_EPS_W : 0.0);
+                const double g = fabs(lu - delta);
+                if (g < *agap) *agap = g;
+                if (!(g >= band)) nr |= NEAR_ACCEPT;
+                if (lu < delta) { next = i; break; }
+                /* rejected: the next child is tested against norm(max(0, P - q)) */
+                double S = 0.0, E = 0.0;
+                for (int v = 0; v < V; ++v) {
+                    const double q = exp(widen(dft, is_bf16, trow + (size_t)v) / T - lse_d);
+                    const double P = wbuf[v] / Sw;
+                    S += fmax(0.0, P - q);
+                    if (P + ebuf[v] / Sw + ORACLE_EPS_W * q > q) E += ebuf[v] / Sw + ORACLE_EPS_W * q;
+                }
+                const double thr_band = level == 0 ? ORACLE_NEAR : ORACLE_NEAR + E;
+                if (fabs(S - ORACLE_RESIDUAL_MIN) < resid_gap) resid_gap = fabs(S - ORACLE_RESIDUAL_MIN);
+                if (fabs(S - ORACLE_RESIDUAL_MIN) < thr_band) nr |= NEAR_CDF;
+                if (S < ORACLE_RESIDUAL_MIN || S != S) {
+                    st = st | ST_RESID0; /* the residual vanished: P stays */
+                    continue;
+                }
+                for (int v = 0; v < V; ++v) {
+                    const double q = exp(widen(dft, is_bf16, trow + (size_t)v) / T - lse_d);
+                    const double P = wbuf[v] / Sw;
+                    const double e = ebuf[v] / Sw + ORACLE_EPS_W * q;
+                    wbuf[v] = fmax(0.0, P - q);
+                    ebuf[v] = (P + ebuf[v] / Sw + ORACLE_EPS_W * q > q) ? e : 0.0;
+                }
+                Sw = S;
+                ++level;
+            }
+            if (next >= 0) {
+                out_nodes[n] = next;
+                ++n;
+                c = next;
+                continue;
+            }
+            /* the extra token: from P (p itself when nothing was rejected) */
+            k = inverse_cdf(wbuf, V, u_res, &nr, cgap);
+            if (resid_gap < *cgap) *cgap = resid_gap;
+            if (level >= 2) {
+                double Et = 0.0;
+                for (int v = 0; v < V; ++v) Et += ebuf[v];
+                if (*cgap < ORACLE_NEAR + Et) nr |= NEAR_CDF;
+            }
+            break;
+        }
+    }
+    if (st & (ST_ROW | ST_TOKEN | ST_UNIFORM | ST_TEMP | ST_TREE)) {
+        for (int i = 0; i < N; ++i) { out_nodes[i] = -1; out_tok[i] = -1; }
+        *out_n = 0;
+        *status = st;
+        *near = 0;
+        return;
+    }
+    for (int j = 0; j < n; ++j) out_tok[j] = tok[out_nodes[j]];
+    out_tok[n] = k;
+    *out_n = n;
+    *status = st;
+    *near = nr;
+}
+
+/*
+ * target, draft: [B][N][V]; parent, tokens, u_accept: [B][N]; keep: [B][N] or
+ * NULL.  Outputs: out_nodes, out_tokens [B][N]; out_n [B]; log_norm [B][2N]
+ * (target rows, then draft rows; NaN for rows not read); row_status, near_tie
+ * [B]; accept_gap, cdf_gap [B] as in sv_oracle_verify.  Returns 0, -1 on a bad
+ * shape (N outside [1, 64], V < 1), -2 if memory ran out.
+ */
+int sv_oracle_tree_verify(const void* target, const void* draft, int is_bf16, const int32_t* parent,
+                          const int32_t* tokens, const int32_t* keep, const float* temperature,
+                          const float* u_accept, const float* u_resample, int B, int N, int V,
+                          int32_t* out_nodes, int32_t* out_tokens, int32_t* out_n, double* log_norm,
+                          int32_t* row_status, int32_t* near_tie, double* accept_gap, double* cdf_gap,
+                          int n_threads)
+{
+    if (B < 0 || N < 1 || N > 64 || V < 1) return -1;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        double* wbuf = (double*)malloc(sizeof(double) * 2 * (size_t)V);
+        if (!wbuf) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b) {
+            if (!wbuf) continue;
+            const size_t o = (size_t)b * N;
+            tree_one(target, draft, is_bf16, parent + o, tokens + o, keep ? keep + o : NULL,
+                     (double)temperature[b], u_accept + o, (double)u_resample[b], N, V, (size_t)b,
+                     out_nodes + o, out_tokens + o, out_n + b, log_norm + 2 * o, row_status + b, near_tie + b,
+                     accept_gap + b, cdf_gap + b, wbuf, wbuf + V);
+        }
+        free(wbuf);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Pruning by cumulative path probability [SpecLA, Metodologia 3, "Poda Guiada
+ * por Confianca": paths of low cumulative draft log-probability are removed
+ * before verification].  For node i >= 1 with parent c:
+ *     cum[i] = cum[c] + log q_c(tok[i]),  cum[0] = 0,
+ * log q_c = ld[c]/T - lse(ld[c]/T) for T > 0; for T == 0 the draft is greedy and
+ * log q_c(x) is 0 at the first argmax of draft row c, -inf elsewhere.
+ * keep[0] = 1; keep[i] = keep[c] and not (cum[i] < threshold).  Where cum cannot
+ * be formed (bad temperature or tree: every node of the sequence; a token
+ * outside [0, V) or a bad draft row c: the node) it is NaN and the node is kept,
+ * so the verification reports the fault.  out_keep [B][N] int32, out_cum [B][N].
+ */
+int sv_oracle_tree_prune(const void* draft, int is_bf16, const int32_t* parent, const int32_t* tokens,
+                         const float* temperature, double threshold, int B, int N, int V, int32_t* out_keep,
+                         double* out_cum)
+{
+    if (B < 0 || N < 1 || N > 64 || V < 1) return -1;
+    for (int b = 0; b < B; ++b) {
+        const size_t o = (size_t)b * N;
+        const int32_t* par = parent + o;
+        const int32_t* tok = tokens + o;
+        const double T = (double)temperature[b];
+        int ok = (T == 0.0 || (isfinite(T) && T >= ORACLE_T_MIN)) && par[0] == -1;
+        for (int i = 1; i < N; ++i)
+            if (par[i] < 0 || par[i] >= i) ok = 0;
+        out_keep[o] = 1;
+        out_cum[o] = ok ? 0.0 : NAN;
+        for (int i = 1; i < N; ++i) {
+            if (!ok) { out_keep[o + i] = 1; out_cum[o + i] = NAN; continue; }
+            const int c = par[i];
+            const size_t row = (o + (size_t)c) * (size_t)V;
+            double lq = NAN;
+            if (tok[i] >= 0 && tok[i] < V) {
+                if (T == 0.0) {
+                    const int a = row_argmax(draft, is_bf16, row, V);
+                    if (a >= 0) lq = (tok[i] == a) ? 0.0 : -INFINITY;
+                } else {
+                    double lse;
+                    if (row_lse(draft, is_bf16, row, V, T, &lse))
+                        lq = widen(draft, is_bf16, row + (size_t)tok[i]) / T - lse;
+                }
+            }
+            out_cum[o + i] = out_cum[o + c] + lq;
+            out_keep[o + i] = out_keep[o + c] && !(out_cum[o + i] < threshold);
+        }
+    }
+    return 0;
+}

@@ -76,6 +76,22 @@ BANDIT_MUTANTS = {
     "bandit_reward_to_arm0": ("N[*arm] += 1.0;\n        R[*arm] += reward;", "N[*arm] += 1.0;\n        R[0] += reward;"),
 }
 
+TREE_MUTANTS = {
+    "tree_residual_sign": ("wbuf[v] = fmax(0.0, P - q);", "wbuf[v] = fmax(0.0, q - P);"),
+    "tree_later_tests_use_p": ("const double lp = level == 0 ?", "const double lp = 1 ?"),
+    "tree_residual_never_applied": ("if (S < ORACLE_RESIDUAL_MIN || S != S) {", "if (1) {"),
+    "tree_keep_ignored": ("in[i] = in[par[i]] && (keep == NULL || keep[i] != 0);", "in[i] = in[par[i]];"),
+    "tree_parent_off_by_one": ("if (par[i] < 0 || par[i] >= i) { st |= ST_TREE;", "if (par[i] < 0 || par[i] > i) { st |= ST_TREE;"),
+    "tree_leaf_draft_row_read": ("if (first >= 0) {\n                if (!row_lse(dft", "if (first >= -1) {\n                if (!row_lse(dft"),
+    "tree_greedy_inverted": ("if (tok[i] == a) { next = i; break; }", "if (tok[i] != a) { next = i; break; }"),
+    "tree_fallback_not_flagged": ("st = st | ST_RESID0; /* the residual vanished: P stays */", "; /* P stays */"),
+    "prune_child_row": ("const size_t row = (o + (size_t)c) * (size_t)V;", "const size_t row = (o + (size_t)i) * (size_t)V;"),
+    # (keep[i] without keep[parent] is an equivalent mutant: log q <= 0, so a path's
+    # cumulative log-probability never rises and a pruned parent's children fall below
+    # the threshold too)
+    "prune_not_cumulative": ("out_cum[o + i] = out_cum[o + c] + lq;", "out_cum[o + i] = lq;"),
+}
+
 BANDIT_SIM_MUTANTS = {
     "sim_gap_from_first_arm": ("if (mu[k] > mu_max) mu_max = mu[k];", ";"),
     "sim_reward_draw_of_last_row": ("reward = (double)us[2 * K] < mu[arm] ? 1 : 0;",
@@ -90,7 +106,7 @@ BANDIT_SIM_MUTANTS = {
 
 def _build_mutant(name, tmpdir):
     src = open(SRC).read()
-    old, new = {**MUTANTS, **TOPF_MUTANTS, **BANDIT_MUTANTS, **BANDIT_SIM_MUTANTS}[name]
+    old, new = {**MUTANTS, **TOPF_MUTANTS, **BANDIT_MUTANTS, **BANDIT_SIM_MUTANTS, **TREE_MUTANTS}[name]
     assert src.count(old) == 1, f"mutation site for {name} not unique"
     path = os.path.join(tmpdir, f"{name}.c")
     with open(path, "w") as f:
@@ -142,6 +158,12 @@ class _OracleWith:
     def cache_lookup(self, *a, **k):
         return oracle.cache_lookup(*a, lib=self.lib, **k)
 
+    def tree_verify(self, *a, **k):
+        return oracle.tree_verify(*a, lib=self.lib, **k)
+
+    def tree_prune(self, *a, **k):
+        return oracle.tree_prune(*a, lib=self.lib, **k)
+
 
 @pytest.mark.parametrize("name", sorted(TOPF_MUTANTS))
 def test_topf_mutant_is_caught(name):
@@ -186,6 +208,22 @@ def test_bandit_sim_mutant_is_caught(name):
             try:
                 check(lambda mu, T, policy, U: oracle.bandit_simulate(mu, T, policy, U, lib=lib, with_state=True),
                       lambda K, policy: oracle.Bandit(K, policy, lib=clean))
+            except Exception as e:  # noqa: BLE001 - any failure counts as caught
+                caught.append((check.__name__, type(e).__name__))
+                break
+        assert caught, f"planted mistake {name} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(TREE_MUTANTS))
+def test_tree_mutant_is_caught(name):
+    import tree_pins as TP
+    with tempfile.TemporaryDirectory() as d:
+        O = _OracleWith(_build_mutant(name, d))
+        caught = []
+        for check in TP.ALL_TREE_CHECKS:
+            try:
+                with np.errstate(all="ignore"):
+                    check(O)
             except Exception as e:  # noqa: BLE001 - any failure counts as caught
                 caught.append((check.__name__, type(e).__name__))
                 break
