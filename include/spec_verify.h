@@ -84,6 +84,7 @@ typedef enum { SV_DTYPE_F32 = 0, SV_DTYPE_BF16 = 1 } sv_dtype;
                                      the token was drawn from p_n instead */
 #define SV_ROW_BAD_UNIFORM 16     /* T > 0 and some u_accept[b][j] or u_resample[b]
                                      outside [0, 1) or NaN */
+#define SV_ROW_BAD_TREE 32        /* spec_verify_tree: a parent index out of range */
 
 /*
  * Bytes of device workspace spec_verify() needs for this shape (0 on a bad
@@ -328,6 +329,82 @@ sv_status spec_verify_bandit_step(const int32_t* n_accepted, int B, int gamma, i
 sv_status spec_verify_bandit_simulate(const double* mu, int K, int T, int policy, int runs,
                                       const float* uniforms, double* out_regret, double* out_state,
                                       struct CUstream_st* stream);
+
+/*
+ * ---------------------------------------------------------------------------
+ * Token trees [SpecLA, Metodologia 1, "Kernels de Verificacao de Topologia
+ * Conscientes": drafts shaped as chains or as branching trees; Metodologia 3,
+ * "Poda Guiada por Confianca": paths of low cumulative draft log-probability are
+ * removed before verification; Speculative Speculative Decoding, "Significado e
+ * Impacto": the method is compatible with token trees].
+ *
+ * Layout of sequence b with N nodes: node 0 is the root (the context verified
+ * so far); node i >= 1 carries a draft token tokens[b][i] and a parent
+ * parent[b][i] in [0, i) (parent[b][0] = -1), so parents come before children.
+ * target_logits [B][N][V] hold the target's next-token logits at node i's
+ * context (the path to i, tokens[b][i] included), draft_logits [B][N][V] the
+ * draft's there (the distribution node i's children were drawn from).
+ */
+#define SV_MAX_TREE_NODES 64
+
+/*
+ * Verify B token trees.  The pages give no rule for several candidates; this is
+ * the multi-candidate form of spec_verify's test (its output law is the
+ * target's when the children of a node are independent draws from q there):
+ * at node c (first the root) P is the target's p at c; the children of c that
+ * take part are tested in increasing index, child i accepted iff
+ *     log u_accept[b][i] < log P(x_i) - log q_c(x_i);
+ * after a rejection P becomes norm(max(0, P - q_c)) (or stays P when that mass
+ * is below 2^-18: status bit SV_ROW_RESIDUAL_ZERO); an accepted child becomes c;
+ * when no child of c is accepted, or c has none, the extra token is drawn from P
+ * by spec_verify's inverse CDF with u_resample[b].  T = 0: the first child whose
+ * token is the first argmax of target row c is accepted, else that argmax is the
+ * extra token.  On a chain (parent i - 1) the result is spec_verify's.
+ *
+ *   keep            optional [B][N] int32: node i >= 1 takes part iff keep != 0
+ *                   and its parent takes part (spec_verify_tree_prune's output)
+ *   u_accept        [B][N] float (entry 0 unused);  u_resample [B] float
+ *   out_nodes       [B][N] int32: the accepted nodes in path order, then -1
+ *   out_tokens      [B][N] int32: their tokens, the extra token, then -1
+ *   out_n_accepted  [B] int32: the number of accepted nodes (path depth)
+ *   out_log_norm    optional [B][2N] double: lse of target row i at [i], of draft
+ *                   row i at [N + i], for the rows the walk read; NaN elsewhere
+ *   out_row_status  optional [B] int32: SV_ROW_* bits.  The walk reads target row
+ *                   c of every node c it visits and (T > 0) draft row c when c has
+ *                   children taking part; status 2 only for a bad row among them.
+ *                   Status 1 / 16 concern the nodes that take part; 32 a parent
+ *                   index out of range.  With 1, 2, 4, 16 or 32 nothing is emitted.
+ *
+ * All pointers are caller-owned device memory (the logits 16-byte aligned);
+ * nothing is allocated and no workspace is needed; one launch (a cluster of up
+ * to 8 CTAs per tree).  Host-checkable errors (N outside [1,
+ * SV_MAX_TREE_NODES], V outside [1, SV_MAX_V], B < 1, a null pointer, a bad
+ * dtype, misalignment) return before any launch.
+ */
+sv_status spec_verify_tree(const void* target_logits, const void* draft_logits, sv_dtype dt,
+                           const int32_t* parent, const int32_t* tokens, const int32_t* keep,
+                           const float* temperature, const float* u_accept, const float* u_resample,
+                           int B, int N, int V, int32_t* out_nodes, int32_t* out_tokens,
+                           int32_t* out_n_accepted, double* out_log_norm, int32_t* out_row_status,
+                           struct CUstream_st* stream);
+
+/*
+ * Pruning by path probability, before verification: for node i >= 1 with parent c
+ *     out_cum[b][i] = out_cum[b][c] + log q_c(tokens[b][i]),  out_cum[b][0] = 0,
+ * log q_c = the draft's log-softmax of row c at temperature T (T = 0: 0 at the
+ * first argmax of draft row c, -inf elsewhere), and
+ *     out_keep[b][i] = out_keep[b][c] and not (out_cum[b][i] < threshold).
+ * Where the sum cannot be formed (a bad temperature or parent index: every node
+ * of the sequence; a token outside [0, V) or a bad draft row: that node and what
+ * adds to it) out_cum is NaN and the node is kept, so spec_verify_tree reports
+ * the fault.  Pruning chooses the proposals: spec_verify_tree's output law is
+ * the target's only for children drawn independently from q, which a
+ * threshold on their own probability is not (greedy trees excepted).
+ *   out_keep [B][N] int32, out_cum [B][N] double.  Two launches.
+ */
+sv_status spec_verify_tree_prune(const void* draft_logits, sv_dtype dt, const int32_t* parent,
+                                 const int32_t* tokens, const float* temperature, double threshold, int B,
+                                 int N, int V, int32_t* out_keep, double* out_cum, struct CUstream_st* stream);
 
 #ifdef __cplusplus
 }

@@ -23,10 +23,12 @@ EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_
             "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc",
             "spec_verify_fanout", "spec_verify_topf", "spec_verify_cache_lookup",
             "spec_verify_bandit_state_size", "spec_verify_bandit_init", "spec_verify_bandit_step",
-            "spec_verify_bandit_simulate")
+            "spec_verify_bandit_simulate", "spec_verify_tree", "spec_verify_tree_prune")
 MAX_TOPF = 32
 MAX_ARMS = 16
 BANDIT_UCB1, BANDIT_THOMPSON = 0, 1
+MAX_TREE_NODES = 64
+ROW_BAD_TREE = 32
 
 _lib = None
 
@@ -72,6 +74,10 @@ def load_library(path: str = LIB_PATH):
     lib.spec_verify_bandit_step.restype = i32
     lib.spec_verify_bandit_simulate.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
     lib.spec_verify_bandit_simulate.restype = i32
+    lib.spec_verify_tree.argtypes = [vp, vp, i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.spec_verify_tree.restype = i32
+    lib.spec_verify_tree_prune.argtypes = [vp, i32, vp, vp, vp, ctypes.c_double, i32, i32, i32, vp, vp, vp]
+    lib.spec_verify_tree_prune.restype = i32
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -313,6 +319,85 @@ def bandit_simulate(mu: torch.Tensor, T: int, policy: int, uniforms: torch.Tenso
                                                   regret.data_ptr(), state.data_ptr() if with_state else None,
                                                   s.cuda_stream))
     return (regret, state) if with_state else regret
+
+
+def tree_verify(target: torch.Tensor, draft: torch.Tensor, parent: torch.Tensor, tokens: torch.Tensor,
+                temperature: torch.Tensor, u_accept: torch.Tensor, u_resample: torch.Tensor,
+                keep: torch.Tensor | None = None, *, return_log_norm: bool = False, return_row_status: bool = False,
+                stream: torch.cuda.Stream | None = None):
+    """Verify B token trees on the GPU (see include/spec_verify.h).
+
+    target, draft [B, N, V] (float32 or bfloat16); parent, tokens, u_accept [B, N];
+    keep [B, N] int32 or None; temperature, u_resample [B].  Returns (out_nodes [B, N],
+    out_tokens [B, N], n_accepted [B]) plus, if asked, log_norm [B, 2N] and row_status [B]."""
+    lib = load_library()
+    if not isinstance(target, torch.Tensor) or target.device.type != "cuda" or target.dim() != 3:
+        raise ValueError("target must be a [B, N, V] CUDA tensor")
+    device = target.device
+    B, N, V = target.shape
+    dt = _dt_code(target.dtype)
+    _check(target, "target", None, (B, N, V), device)
+    _check(draft, "draft", target.dtype, (B, N, V), device)
+    for name, t in (("parent", parent), ("tokens", tokens)):
+        _check(t, name, torch.int32, (B, N), device)
+    if keep is not None:
+        _check(keep, "keep", torch.int32, (B, N), device)
+    _check(temperature, "temperature", torch.float32, (B,), device)
+    _check(u_accept, "u_accept", torch.float32, (B, N), device)
+    _check(u_resample, "u_resample", torch.float32, (B,), device)
+    nodes = torch.empty((B, N), dtype=torch.int32, device=device)
+    toks = torch.empty((B, N), dtype=torch.int32, device=device)
+    n = torch.empty((B,), dtype=torch.int32, device=device)
+    log_norm = torch.empty((B, 2 * N), dtype=torch.float64, device=device) if return_log_norm else None
+    status = torch.empty((B,), dtype=torch.int32, device=device) if return_row_status else None
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_tree(target.data_ptr(), draft.data_ptr(), dt, parent.data_ptr(), tokens.data_ptr(),
+                                       keep.data_ptr() if keep is not None else None, temperature.data_ptr(),
+                                       u_accept.data_ptr(), u_resample.data_ptr(), B, N, V, nodes.data_ptr(),
+                                       toks.data_ptr(), n.data_ptr(),
+                                       log_norm.data_ptr() if log_norm is not None else None,
+                                       status.data_ptr() if status is not None else None, s.cuda_stream))
+    out = (nodes, toks, n)
+    if return_log_norm:
+        out += (log_norm,)
+    if return_row_status:
+        out += (status,)
+    return out
+
+
+def tree_prune(draft: torch.Tensor, parent: torch.Tensor, tokens: torch.Tensor, temperature: torch.Tensor,
+               threshold: float, *, stream: torch.cuda.Stream | None = None):
+    """Cumulative draft log-probability of every node and the keep mask at
+    ``threshold``: (keep [B, N] int32, cum [B, N] float64), on the GPU."""
+    lib = load_library()
+    device = draft.device
+    B, N, V = draft.shape
+    dt = _dt_code(draft.dtype)
+    _check(draft, "draft", None, (B, N, V), device)
+    _check(parent, "parent", torch.int32, (B, N), device)
+    _check(tokens, "tokens", torch.int32, (B, N), device)
+    _check(temperature, "temperature", torch.float32, (B,), device)
+    keep = torch.empty((B, N), dtype=torch.int32, device=device)
+    cum = torch.empty((B, N), dtype=torch.float64, device=device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_tree_prune(draft.data_ptr(), dt, parent.data_ptr(), tokens.data_ptr(),
+                                             temperature.data_ptr(), float(threshold), B, N, V, keep.data_ptr(),
+                                             cum.data_ptr(), s.cuda_stream))
+    return keep, cum
+
+
+def tree_to_device(w, device="cuda"):
+    """Copy a ``workloads.TreeWorkload`` (numpy) to torch tensors on ``device``."""
+    def logits(a):
+        t = torch.from_numpy(a)
+        if w.dtype == "bf16":
+            t = t.view(torch.bfloat16)
+        return t.to(device)
+    return dict(target=logits(w.target), draft=logits(w.draft), parent=torch.from_numpy(w.parent).to(device),
+                tokens=torch.from_numpy(w.tokens).to(device), temperature=torch.from_numpy(w.temperature).to(device),
+                u_accept=torch.from_numpy(w.u_accept).to(device), u_resample=torch.from_numpy(w.u_resample).to(device))
 
 
 def to_device(w, device="cuda"):

@@ -31,6 +31,7 @@
 #include "sv_small.cuh"
 #include "sv_topf.cuh"
 #include "sv_bandit.cuh"
+#include "sv_tree.cuh"
 
 namespace {
 
@@ -679,5 +680,108 @@ extern "C" sv_status spec_verify_bandit_simulate(const double* mu, int K, int T,
     const unsigned grid = (unsigned)cdiv(runs, kRunsPerCta);
     sv::sv_bandit_simulate<<<grid, sv::kBanditSimThreads, 0, (cudaStream_t)stream>>>(mu, K, T, policy, runs, uniforms,
                                                                                        out_regret, out_state);
+    return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------- token trees
+
+static_assert(sv::kTreeMaxNodes == SV_MAX_TREE_NODES, "tree node limit");
+
+namespace {
+
+// Groups of 16 bytes per row, and the cluster split: enough CTAs per tree to
+// spread a row over several SMs, as long as the whole batch stays resident (two
+// 512-thread CTAs per SM), and at least 512 groups (one per thread) per CTA.
+void tree_plan(int B, int V, int esz, int* CL, long long* G, long long* GPC, long long* GPW)
+{
+    const int vec = 16 / esz;
+    *G = cdiv(V, vec);
+    int cl = 1;
+    while (cl < sv::kTreeMaxCluster && (long long)B * cl * 2 <= 2LL * kSmCount &&
+           *G / (cl * 2) >= sv::kTreeThreads)
+        cl *= 2;
+    *CL = cl;
+    *GPC = cdiv(*G, cl);
+    *GPW = cdiv(cdiv(*GPC, sv::kTreeWarps), 32) * 32;
+}
+
+}  // namespace
+
+extern "C" sv_status spec_verify_tree(const void* target_logits, const void* draft_logits, sv_dtype dt,
+                                      const int32_t* parent, const int32_t* tokens, const int32_t* keep,
+                                      const float* temperature, const float* u_accept, const float* u_resample,
+                                      int B, int N, int V, int32_t* out_nodes, int32_t* out_tokens,
+                                      int32_t* out_n_accepted, double* out_log_norm, int32_t* out_row_status,
+                                      struct CUstream_st* stream)
+{
+    if (dt != SV_DTYPE_F32 && dt != SV_DTYPE_BF16) return SV_ERR_UNSUPPORTED_DTYPE;
+    if (B < 1 || N < 1 || N > SV_MAX_TREE_NODES || V < 1 || V > SV_MAX_V) return SV_ERR_INVALID_ARG;
+    if (!target_logits || !draft_logits || !parent || !tokens || !temperature || !u_accept || !u_resample ||
+        !out_nodes || !out_tokens || !out_n_accepted)
+        return SV_ERR_INVALID_ARG;
+    if (!aligned(target_logits, 16) || !aligned(draft_logits, 16) || !aligned(parent, 4) || !aligned(tokens, 4) ||
+        !aligned(keep, 4) || !aligned(temperature, 4) || !aligned(u_accept, 4) || !aligned(u_resample, 4) ||
+        !aligned(out_nodes, 4) || !aligned(out_tokens, 4) || !aligned(out_n_accepted, 4) ||
+        !aligned(out_log_norm, 8) || !aligned(out_row_status, 4))
+        return SV_ERR_MISALIGNED;
+    const int esz = dt == SV_DTYPE_BF16 ? 2 : 4;
+    sv::TreeArgs g;
+    g.tgt = target_logits; g.dft = draft_logits; g.parent = parent; g.tokens = tokens; g.keep = keep;
+    g.temperature = temperature; g.u_accept = u_accept; g.u_resample = u_resample;
+    g.out_nodes = out_nodes; g.out_tokens = out_tokens; g.out_n = out_n_accepted;
+    g.out_log_norm = out_log_norm; g.out_status = out_row_status;
+    g.N = N; g.V = V;
+    int CL;
+    tree_plan(B, V, esz, &CL, &g.G, &g.GPC, &g.GPW);
+    const bool vec16 = ((long long)V * esz) % 16 == 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((long long)B * CL));
+    cfg.blockDim = dim3(sv::kTreeThreads);
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (dt == SV_DTYPE_BF16)
+        e = vec16 ? cudaLaunchKernelEx(&cfg, sv::sv_tree<2, true>, g) : cudaLaunchKernelEx(&cfg, sv::sv_tree<2, false>, g);
+    else
+        e = vec16 ? cudaLaunchKernelEx(&cfg, sv::sv_tree<4, true>, g) : cudaLaunchKernelEx(&cfg, sv::sv_tree<4, false>, g);
+    return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+extern "C" sv_status spec_verify_tree_prune(const void* draft_logits, sv_dtype dt, const int32_t* parent,
+                                            const int32_t* tokens, const float* temperature, double threshold,
+                                            int B, int N, int V, int32_t* out_keep, double* out_cum,
+                                            struct CUstream_st* stream)
+{
+    if (dt != SV_DTYPE_F32 && dt != SV_DTYPE_BF16) return SV_ERR_UNSUPPORTED_DTYPE;
+    if (B < 1 || N < 1 || N > SV_MAX_TREE_NODES || V < 1 || V > SV_MAX_V || threshold != threshold)
+        return SV_ERR_INVALID_ARG;
+    if (!draft_logits || !parent || !tokens || !temperature || !out_keep || !out_cum) return SV_ERR_INVALID_ARG;
+    if (!aligned(draft_logits, 16) || !aligned(parent, 4) || !aligned(tokens, 4) || !aligned(temperature, 4) ||
+        !aligned(out_keep, 4) || !aligned(out_cum, 8))
+        return SV_ERR_MISALIGNED;
+    const int esz = dt == SV_DTYPE_BF16 ? 2 : 4;
+    sv::PruneArgs g;
+    g.dft = draft_logits; g.parent = parent; g.tokens = tokens; g.temperature = temperature;
+    g.threshold = threshold; g.out_keep = out_keep; g.out_cum = out_cum;
+    g.B = B; g.N = N; g.V = V;
+    g.G = cdiv(V, 16 / esz);
+    const bool vec16 = ((long long)V * esz) % 16 == 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    const unsigned grid = (unsigned)((long long)B * N);
+    if (dt == SV_DTYPE_BF16) {
+        if (vec16) sv::sv_tree_prune_rows<2, true><<<grid, sv::kPruneThreads, 0, st>>>(g);
+        else sv::sv_tree_prune_rows<2, false><<<grid, sv::kPruneThreads, 0, st>>>(g);
+    } else {
+        if (vec16) sv::sv_tree_prune_rows<4, true><<<grid, sv::kPruneThreads, 0, st>>>(g);
+        else sv::sv_tree_prune_rows<4, false><<<grid, sv::kPruneThreads, 0, st>>>(g);
+    }
+    if (cudaGetLastError() != cudaSuccess) return SV_ERR_CUDA;
+    sv::sv_tree_prune_walk<<<(unsigned)cdiv(B, 128), 128, 0, st>>>(g);
     return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }

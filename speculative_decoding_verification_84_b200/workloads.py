@@ -268,3 +268,85 @@ def bandit_uniforms(runs: int, T: int, K: int, seed: int) -> np.ndarray:
     for r in range(runs):
         out[r] = draw_uniforms(_rng(seed, 7, r), (T + 1, 2 * K + 1))
     return out
+
+
+# ----------------------------------------------------------------------------- token trees
+
+@dataclasses.dataclass
+class TreeWorkload:
+    """One batch of tree-verification inputs (host numpy arrays).
+
+    target, draft: [B, N, V] (float32, or uint16 bf16 bits): the next-token logits
+    at node i's context; parent, tokens, u_accept: [B, N] (node 0 is the root:
+    parent -1, token and uniform unused); temperature, u_resample: [B]."""
+
+    name: str
+    dtype: str
+    target: np.ndarray
+    draft: np.ndarray
+    parent: np.ndarray
+    tokens: np.ndarray
+    temperature: np.ndarray
+    u_accept: np.ndarray
+    u_resample: np.ndarray
+
+    @property
+    def B(self):
+        return self.target.shape[0]
+
+    @property
+    def N(self):
+        return self.target.shape[1]
+
+    @property
+    def V(self):
+        return self.target.shape[2]
+
+
+def tree_parents(branching: Sequence[int]) -> np.ndarray:
+    """Parent array of a tree in breadth-first order: the root has branching[0]
+    children, each of those branching[1], and so on (so parent[i] < i)."""
+    par, level = [-1], [0]
+    for k in branching:
+        nxt = []
+        for p in level:
+            for _ in range(int(k)):
+                par.append(p)
+                nxt.append(len(par) - 1)
+        level = nxt
+    return np.asarray(par, dtype=np.int32)
+
+
+def make_tree(B: int, branching: Sequence[int], V: int, dtype: str, *, seed: int, T=1.0, rho: float = 0.9,
+              name: Optional[str] = None) -> TreeWorkload:
+    """A batch of token trees of one shape, built like c3: every node's target
+    row N(0, 3^2) + a Zipf(1.1) log-bias over a permutation shared by the batch,
+    its draft row rho * target + sqrt(1 - rho^2) * N(0, 3^2).  Node i's token is
+    drawn from softmax(draft row of its parent / T) (T = 1 for greedy sequences,
+    so siblings differ), independently for every sibling.  T may be a scalar or
+    a sequence, repeated over the batch.  Each sequence has its own streams (key
+    8, b)."""
+    par = tree_parents(branching)
+    N = par.size
+    temp = np.resize(np.asarray(T, dtype=np.float32).reshape(-1), B).astype(np.float32)
+    bias = zipf_log_bias(V, _rng(seed, 8, 1 << 20).permutation(V))
+    dt = np.uint16 if dtype == "bf16" else np.float32
+    tgt = np.empty((B, N, V), dt)
+    dft = np.empty((B, N, V), dt)
+    tok = np.zeros((B, N), np.int32)
+    for b in range(B):
+        rng = _rng(seed, 8, b)
+        t64 = rng.standard_normal((N, V)) * 3.0 + bias
+        d64 = rho * t64 + math.sqrt(1.0 - rho * rho) * 3.0 * rng.standard_normal((N, V))
+        tgt[b] = _store(t64, dtype)
+        dft[b] = _store(d64, dtype)
+        dstored = _stored_to_f64(dft[b], dtype)
+        Tb = float(temp[b]) if temp[b] > 0 else 1.0
+        gu = np.clip(rng.random((N, V)), 1e-300, 1.0 - 2.0 ** -53)
+        for i in range(1, N):
+            tok[b, i] = gumbel_max_tokens(dstored[par[i]][None], Tb, gu[i][None])[0]
+    urng = _rng(seed, 8, (1 << 20) + 1)
+    ua = draw_uniforms(urng, (B, N))
+    ur = draw_uniforms(urng, (B,))
+    label = name or f"tree_{B}x{'-'.join(map(str, branching))}x{V}_{dtype}"
+    return TreeWorkload(label, dtype, tgt, dft, np.tile(par, (B, 1)), tok, temp, ua, ur)
