@@ -428,6 +428,87 @@ def bandit_row_line(w, dev, lib, binding, cpu_seconds=2.0):
     return out
 
 
+TREE_SHAPE = (3, 2, 1)  # 16 nodes: 3 candidates, 2 continuations each, then 1
+
+
+def tree_row_line(dev, lib, binding, peak, peak_kind, cpu_seconds=2.0):
+    """Token-tree verification on B = 64 trees of shape (3, 2, 1) over V = 128256
+    (bf16, built like c3): spec_verify_tree and spec_verify_tree_prune (threshold
+    -12), each timed as CUDA graph replays rotating over input copies whose
+    visited rows exceed 2x L2 in total.  Algorithmic bytes of a verification: the
+    rows the walks read (target row of every visited node, draft row of every
+    visited node with children), counted from its outputs; of the pruning: the
+    draft rows of every node with children."""
+    import torch
+    from speculative_decoding_verification_84_b200 import workloads as W
+    import oracle
+    w = W.make_tree(64, TREE_SHAPE, 128256, "bf16", seed=91, name="t3")
+    base = binding.tree_to_device(w, dev)
+    B, N, V = w.B, w.N, w.V
+    n_copies = 4
+    sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_copies - 1)]
+    stream = torch.cuda.Stream(dev)
+    outs = [torch.empty((B, N), dtype=torch.int32, device=dev) for _ in range(2)] + \
+        [torch.empty((B,), dtype=torch.int32, device=dev)]
+    keep = torch.empty((B, N), dtype=torch.int32, device=dev)
+    cum = torch.empty((B, N), dtype=torch.float64, device=dev)
+
+    def verify(i):
+        d = sets[i % n_copies]
+        rc = lib.spec_verify_tree(d["target"].data_ptr(), d["draft"].data_ptr(), 1, d["parent"].data_ptr(),
+                                  d["tokens"].data_ptr(), None, d["temperature"].data_ptr(), d["u_accept"].data_ptr(),
+                                  d["u_resample"].data_ptr(), B, N, V, outs[0].data_ptr(), outs[1].data_ptr(),
+                                  outs[2].data_ptr(), None, None, stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(binding.status_string(rc))
+
+    def prune(i):
+        d = sets[i % n_copies]
+        rc = lib.spec_verify_tree_prune(d["draft"].data_ptr(), 1, d["parent"].data_ptr(), d["tokens"].data_ptr(),
+                                        d["temperature"].data_ptr(), -12.0, B, N, V, keep.data_ptr(), cum.data_ptr(),
+                                        stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(binding.status_string(rc))
+
+    with torch.cuda.stream(stream):
+        for i in range(4):
+            verify(i)
+            prune(i)
+    torch.cuda.synchronize()
+    ms_v = graph_ms(stream, verify, 400, n_copies)
+    ms_p = graph_ms(stream, prune, 400, n_copies)
+    # the rows the walks read, from the outputs of one verification
+    with torch.cuda.stream(stream):
+        verify(0)
+    torch.cuda.synchronize()
+    nodes, n = outs[0].cpu().numpy(), outs[2].cpu().numpy()
+    par = w.parent[0]
+    has_kids = np.zeros(N, bool)
+    has_kids[par[1:]] = True
+    rows = 0
+    for b in range(B):
+        visited = [0] + [int(x) for x in nodes[b, :n[b]]]
+        rows += len(visited) + int(sum(has_kids[c] for c in visited))
+    alg = rows * V * 2
+    alg_p = B * int(has_kids.sum()) * V * 2
+    gbs, gbs_p = alg / (ms_v / 1e3) / 1e9, alg_p / (ms_p / 1e3) / 1e9
+    # the oracle on the same batch, for comparison
+    t0, reps = time.perf_counter(), 0
+    while time.perf_counter() - t0 < cpu_seconds or reps == 0:
+        oracle.tree_verify(w.target, w.draft, w.parent, w.tokens, w.temperature, w.u_accept, w.u_resample, bf16=True)
+        reps += 1
+    cpu_s = (time.perf_counter() - t0) / reps
+    return {"workload": "t3: B=64 trees (3,2,1) = 16 nodes, V=128256, bf16, rho 0.9, T=1",
+            "us_per_call_verify": 1e3 * ms_v, "trees_per_s": B / (ms_v / 1e3),
+            "mean_accepted": float(n.mean()), "rows_read": rows, "algorithmic_bytes_verify": alg,
+            "hbm_gbs_verify": gbs, "frac_of_peak_verify": gbs / peak,
+            "us_per_call_prune": 1e3 * ms_p, "algorithmic_bytes_prune": alg_p, "hbm_gbs_prune": gbs_p,
+            "frac_of_peak_prune": gbs_p / peak, "peak_source": peak_kind,
+            "l2": f"{n_copies} input copies rotated ({n_copies * 2 * w.target.nbytes / 1e6:.0f} MB)",
+            "cpu_baseline": {"kind": "oracle", "cores": oracle.max_threads(), "trees_per_s": B / cpu_s,
+                             "sample": f"{reps} passes over the 64 trees"}}
+
+
 def cache_row_line(w, dev, lib, binding, peak, peak_kind, budget_ms=20.0):
     """The speculation-cache row on one workload: spec_verify_topf with the
     geometric fan-out of a 64-slot budget at acceptance rate 0.7 (then at most 32
@@ -615,6 +696,8 @@ def run_ours(args):
         torch.cuda.empty_cache()
         per_config["bandit_row_c3"] = bandit_row_line(W.make_workload(WORKLOAD), dev, lib, binding)
         torch.cuda.empty_cache()
+        per_config["tree_row_t3"] = tree_row_line(dev, lib, binding, peak, peak_kind)
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -671,12 +754,22 @@ def c_copies(w):
 
 
 def run_profile(args):
-    """--profile NAME: warm-up plus K plain calls of workload NAME (c1..c5) and
-    nothing else, so a profiler sees only that workload's launches; no JSON line."""
+    """--profile NAME: warm-up plus K plain calls of workload NAME (c1..c5, or t3:
+    spec_verify_tree on the tree workload) and nothing else, so a profiler sees
+    only that workload's launches; no JSON line."""
     import torch
     from speculative_decoding_verification_84_b200 import binding, build, workloads as W
     build.build()
     lib = binding.load_library()
+    if args.profile == "t3":
+        w = W.make_tree(64, TREE_SHAPE, 128256, "bf16", seed=91, name="t3")
+        d = binding.tree_to_device(w, "cuda:0")
+        for i in range(args.warmup + args.steps):
+            binding.tree_verify(d["target"], d["draft"], d["parent"], d["tokens"], d["temperature"], d["u_accept"],
+                                d["u_resample"])
+        torch.cuda.synchronize()
+        print(f"t3: {args.warmup + args.steps} calls, 1 launch each", flush=True)
+        return 0
     c = Caller(W.make_workload(args.profile), torch.device("cuda", 0), lib, binding)
     for i in range(args.warmup + args.steps):
         c.call(i)
@@ -694,7 +787,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="skip the line's per-workload numbers")
-    ap.add_argument("--profile", choices=PER_CONFIG, default=None,
+    ap.add_argument("--profile", choices=list(PER_CONFIG) + ["t3"], default=None,
                     help="only make warm-up + K calls of this workload (for a profiler); no JSON line")
     args = ap.parse_args()
     if args.profile:
