@@ -67,6 +67,11 @@ def load_library(path: str):
     lib.sv_oracle_tree_prune.argtypes = [p, ctypes.c_int, p, p, p, ctypes.c_double, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, p, p]
     lib.sv_oracle_tree_prune.restype = ctypes.c_int
+    lib.sv_oracle_gemm_bf16.argtypes = [p, p, ctypes.c_int, ctypes.c_int, ctypes.c_int, p]
+    lib.sv_oracle_gemm_bf16.restype = ctypes.c_int
+    lib.sv_oracle_lowrank_head.argtypes = [p, p, p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, p, p, p,
+                                           p]
+    lib.sv_oracle_lowrank_head.restype = ctypes.c_int
     return lib
 
 
@@ -294,3 +299,38 @@ def tree_prune(draft, parent, tokens, temperature, threshold: float, *, bf16: bo
                                 B, N, V, _ptr(keep), _ptr(cum)) != 0:
         raise ValueError("bad tree shape")
     return keep, cum
+
+
+def gemm_bf16(A, B, lib=None) -> np.ndarray:
+    """A [M, K] @ B [N, K]^T over bf16 bit patterns (uint16), in fp64."""
+    lib = _load() if lib is None else lib
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape == (N, K)
+    out = np.empty((M, N), np.float64)
+    if lib.sv_oracle_gemm_bf16(_ptr(A), _ptr(B), M, N, K, _ptr(out)) != 0:
+        raise ValueError("bad shape")
+    return out
+
+
+def lowrank_head(h, w_down, w_up, temperature=None, lib=None):
+    """The low-rank draft head (``sv_oracle_lowrank_head``): (u [M, r] bf16 bits,
+    z [M, V] fp64, lse [M] of bf16(z) / T)."""
+    lib = _load() if lib is None else lib
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    w_down = np.ascontiguousarray(w_down, dtype=np.uint16)
+    w_up = np.ascontiguousarray(w_up, dtype=np.uint16)
+    M, d = h.shape
+    r = w_down.shape[0]
+    V = w_up.shape[0]
+    assert w_down.shape == (r, d) and w_up.shape == (V, r)
+    T = None if temperature is None else np.ascontiguousarray(temperature, dtype=np.float32).reshape(M)
+    u = np.empty((M, r), np.uint16)
+    z = np.empty((M, V), np.float64)
+    lse = np.empty(M, np.float64)
+    if lib.sv_oracle_lowrank_head(_ptr(h), _ptr(w_down), _ptr(w_up), M, d, r, V, None if T is None else _ptr(T),
+                                  _ptr(u), _ptr(z), _ptr(lse)) != 0:
+        raise ValueError("bad shape")
+    return u, z, lse

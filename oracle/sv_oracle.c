@@ -856,3 +856,89 @@ int sv_oracle_tree_prune(const void* draft, int is_bf16, const int32_t* parent, 
     }
     return 0;
 }
+
+/*
+ * The low-rank draft head [SlimSpec, Metodologia, "Arquitetura": z = W_up W_down h
+ * with W_down in R^{r x d}, W_up in R^{V x r}, r << d, instead of W_full h].
+ *
+ * Inputs are bf16 (uint16 bit patterns): h [M][d] (one row per draft position),
+ * W_down [r][d], W_up [V][r].  The product is taken in two contractions, the
+ * intermediate stored in bf16 (this library's reading: the second contraction
+ * takes bf16 operands like the first):
+ *     u[m][i] = bf16( sum_k W_down[i][k] h[m][k] )       (round to nearest even)
+ *     z[m][v] = sum_i W_up[v][i] u[m][i]                  (exact here, fp64)
+ * and the draft row's log-normaliser at temperature T_m of the logits as the
+ * verifier reads them, bf16(z):
+ *     lse[m] = M/T + log sum_v exp((bf16(z[m][v]) - M)/T),  M = max_v bf16(z[m][v])
+ * (NaN for T_m = 0).  Sums of products are accumulated in fp64.
+ */
+/* x rounded to the nearest bf16 value (8 significant bits, the exponent range of
+ * float32), ties to even; +-inf past the largest finite bf16. */
+static double bf16_round(double x)
+{
+    if (!isfinite(x) || x == 0.0) return x;
+    const double tiny = 0x1p-126; /* below it bf16 values are spaced 2^-133 */
+    double r;
+    if (fabs(x) < tiny) {
+        r = ldexp(nearbyint(ldexp(x, 133)), -133);
+    } else {
+        int e;
+        const double f = frexp(x, &e);                /* x = f 2^e, 0.5 <= |f| < 1 */
+        r = ldexp(nearbyint(ldexp(f, 8)), e - 8);     /* default mode: nearest, ties to even */
+    }
+    if (fabs(r) > 0x1.fep127) r = copysign(INFINITY, r);
+    return r;
+}
+
+static double bf16_value(const uint16_t* p, size_t i)
+{
+    uint32_t bits = (uint32_t)p[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* out[m][n] = sum_k A[m][k] B[n][k] over bf16 inputs, in fp64. */
+int sv_oracle_gemm_bf16(const uint16_t* A, const uint16_t* B, int M, int N, int K, double* out)
+{
+    if (M < 0 || N < 0 || K < 0) return -1;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int k = 0; k < K; ++k) s += bf16_value(A, (size_t)m * K + k) * bf16_value(B, (size_t)n * K + k);
+            out[(size_t)m * N + n] = s;
+        }
+    return 0;
+}
+
+/* bf16 of a double, ties to even, as the bit pattern. */
+static uint16_t bf16_bits(double x)
+{
+    const float f = (float)bf16_round(x); /* exact: 8 significant bits fit in float */
+    uint32_t bits;
+    memcpy(&bits, &f, sizeof bits);
+    return (uint16_t)(bits >> 16);
+}
+
+int sv_oracle_lowrank_head(const uint16_t* h, const uint16_t* w_down, const uint16_t* w_up, int M, int d, int r,
+                           int V, const float* temperature, uint16_t* out_u, double* out_z, double* out_lse)
+{
+    if (M < 0 || d < 1 || r < 1 || V < 1) return -1;
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)(M > 0 ? M : 1) * (size_t)r);
+    if (!tmp) return -2;
+    sv_oracle_gemm_bf16(h, w_down, M, r, d, tmp);
+    for (size_t i = 0; i < (size_t)M * r; ++i) out_u[i] = bf16_bits(tmp[i]);
+    free(tmp);
+    sv_oracle_gemm_bf16(out_u, w_up, M, V, r, out_z);
+    for (int m = 0; m < M; ++m) {
+        const double T = temperature ? (double)temperature[m] : 1.0;
+        if (!(T > 0.0) || !isfinite(T)) { out_lse[m] = NAN; continue; }
+        const double* z = out_z + (size_t)m * V;
+        double mx = -INFINITY;
+        for (int v = 0; v < V; ++v) mx = fmax(mx, bf16_round(z[v]));
+        double s = 0.0;
+        for (int v = 0; v < V; ++v) s += exp((bf16_round(z[v]) - mx) / T);
+        out_lse[m] = mx / T + log(s);
+    }
+    return 0;
+}

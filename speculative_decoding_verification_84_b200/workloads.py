@@ -350,3 +350,32 @@ def make_tree(B: int, branching: Sequence[int], V: int, dtype: str, *, seed: int
     ur = draw_uniforms(urng, (B,))
     label = name or f"tree_{B}x{'-'.join(map(str, branching))}x{V}_{dtype}"
     return TreeWorkload(label, dtype, tgt, dft, np.tile(par, (B, 1)), tok, temp, ua, ur)
+
+
+# ----------------------------------------------------------------------------- low-rank draft head
+
+@dataclasses.dataclass
+class LowRankWorkload:
+    """Inputs of the low-rank draft head z = W_up (W_down h), as bf16 bit
+    patterns: h [M, d], w_down [r, d], w_up [V, r]; temperature [M] (the draft
+    position's sequence temperature)."""
+
+    name: str
+    h: np.ndarray
+    w_down: np.ndarray
+    w_up: np.ndarray
+    temperature: np.ndarray
+
+
+def make_lowrank(M: int, d: int, r: int, V: int, *, seed: int, scale: float = 3.0, T=1.0,
+                 name: Optional[str] = None) -> LowRankWorkload:
+    """Random-initialised head (no trained weights here): h ~ N(0, 1),
+    W_down ~ N(0, 1/d), W_up ~ N(0, scale^2 / r), so u = W_down h has unit variance
+    and the logits z have standard deviation about ``scale`` (3, as the target
+    logits of c3).  T may be a scalar or a sequence, repeated over the rows."""
+    rng = _rng(seed, 9)
+    h = f32_to_bf16_bits(rng.standard_normal((M, d)).astype(np.float32))
+    wd = f32_to_bf16_bits((rng.standard_normal((r, d)) / math.sqrt(d)).astype(np.float32))
+    wu = f32_to_bf16_bits((rng.standard_normal((V, r)) * (scale / math.sqrt(r))).astype(np.float32))
+    temp = np.resize(np.asarray(T, dtype=np.float32).reshape(-1), M).astype(np.float32)
+    return LowRankWorkload(name or f"lowrank_{M}x{d}x{r}x{V}", h, wd, wu, temp)

@@ -92,6 +92,13 @@ TREE_MUTANTS = {
     "prune_not_cumulative": ("out_cum[o + i] = out_cum[o + c] + lq;", "out_cum[o + i] = lq;"),
 }
 
+LOWRANK_MUTANTS = {
+    "lowrank_truncates": ("r = ldexp(nearbyint(ldexp(f, 8)), e - 8);", "r = ldexp(trunc(ldexp(f, 8)), e - 8);"),
+    "gemm_b_transposed": ("bf16_value(B, (size_t)n * K + k)", "bf16_value(B, (size_t)k * N + n)"),
+    "lowrank_lse_unrounded": ("s += exp((bf16_round(z[v]) - mx) / T);", "s += exp((z[v] - mx) / T);"),
+    "lowrank_lse_no_temperature": ("out_lse[m] = mx / T + log(s);", "out_lse[m] = mx + log(s);"),
+}
+
 BANDIT_SIM_MUTANTS = {
     "sim_gap_from_first_arm": ("if (mu[k] > mu_max) mu_max = mu[k];", ";"),
     "sim_reward_draw_of_last_row": ("reward = (double)us[2 * K] < mu[arm] ? 1 : 0;",
@@ -106,7 +113,7 @@ BANDIT_SIM_MUTANTS = {
 
 def _build_mutant(name, tmpdir):
     src = open(SRC).read()
-    old, new = {**MUTANTS, **TOPF_MUTANTS, **BANDIT_MUTANTS, **BANDIT_SIM_MUTANTS, **TREE_MUTANTS}[name]
+    old, new = {**MUTANTS, **TOPF_MUTANTS, **BANDIT_MUTANTS, **BANDIT_SIM_MUTANTS, **TREE_MUTANTS, **LOWRANK_MUTANTS}[name]
     assert src.count(old) == 1, f"mutation site for {name} not unique"
     path = os.path.join(tmpdir, f"{name}.c")
     with open(path, "w") as f:
@@ -163,6 +170,12 @@ class _OracleWith:
 
     def tree_prune(self, *a, **k):
         return oracle.tree_prune(*a, lib=self.lib, **k)
+
+    def gemm_bf16(self, *a, **k):
+        return oracle.gemm_bf16(*a, lib=self.lib, **k)
+
+    def lowrank_head(self, *a, **k):
+        return oracle.lowrank_head(*a, lib=self.lib, **k)
 
 
 @pytest.mark.parametrize("name", sorted(TOPF_MUTANTS))
@@ -221,6 +234,22 @@ def test_tree_mutant_is_caught(name):
         O = _OracleWith(_build_mutant(name, d))
         caught = []
         for check in TP.ALL_TREE_CHECKS:
+            try:
+                with np.errstate(all="ignore"):
+                    check(O)
+            except Exception as e:  # noqa: BLE001 - any failure counts as caught
+                caught.append((check.__name__, type(e).__name__))
+                break
+        assert caught, f"planted mistake {name} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(LOWRANK_MUTANTS))
+def test_lowrank_mutant_is_caught(name):
+    import lowrank_pins as LP
+    with tempfile.TemporaryDirectory() as d:
+        O = _OracleWith(_build_mutant(name, d))
+        caught = []
+        for check in LP.ALL_LOWRANK_CHECKS:
             try:
                 with np.errstate(all="ignore"):
                     check(O)
