@@ -406,6 +406,48 @@ sv_status spec_verify_tree_prune(const void* draft_logits, sv_dtype dt, const in
                                  const int32_t* tokens, const float* temperature, double threshold, int B,
                                  int N, int V, int32_t* out_keep, double* out_cum, struct CUstream_st* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * The low-rank draft head [SlimSpec, Metodologia, "Arquitetura": the draft's LM
+ * head z = W_up W_down h with W_down in R^{r x d} and W_up in R^{V x r}, r << d
+ * (e.g. d/8), in place of the full-rank W_full h], producing the draft logits the
+ * verifier reads, on the tensor cores (tcgen05, bf16 in, fp32 accumulation).
+ *
+ * All matrices are bf16, row-major, K-major as stored:
+ *   h [M][d] (one row per draft position: M = B * gamma), W_down [r][d],
+ *   W_up [V][r]; d and r multiples of 8; every pointer 16-byte aligned.
+ *   u [M][r] = bf16(h W_down^T)   (the intermediate is rounded to bf16: the
+ *                                  second contraction takes bf16 operands)
+ *   z [M][V] = bf16(u W_up^T)     (the draft logits)
+ *   out_lse [M] (optional): the log-normaliser of each row of z at temperature
+ *   temperature[m] (null: 1), the value spec_verify's out_log_norm gives for that
+ *   draft row; NaN for T = 0 or an invalid T, and for a row with NaN or +inf.
+ * out_error (optional, device int32): set to 1 if a kernel gave up waiting on its
+ * own pipeline (outputs are then undefined); never set on a working GPU.
+ * Host-checkable errors return before any launch.
+ */
+
+/* Workspace bytes of spec_verify_lowrank_head (u and the normaliser partials);
+ * spec_verify_lowrank_up needs lowrank_workspace_size minus the u part, only when
+ * out_lse is requested.  0 on a bad shape. */
+size_t spec_verify_lowrank_workspace_size(int M, int r, int V);
+
+/* u = bf16(h W_down^T): [M][r]. */
+sv_status spec_verify_lowrank_down(const void* h, const void* w_down, int M, int d, int r, void* out_u,
+                                   int32_t* out_error, struct CUstream_st* stream);
+
+/* z = bf16(u W_up^T): [M][V], and (if out_lse) each row's log-normaliser; the
+ * workspace (256-byte aligned) holds M * ceil(V / 256) partials of 16 bytes. */
+sv_status spec_verify_lowrank_up(const void* u, const void* w_up, int M, int r, int V, const float* temperature,
+                                 void* out_logits, double* out_lse, void* workspace, size_t workspace_bytes,
+                                 int32_t* out_error, struct CUstream_st* stream);
+
+/* Both contractions: the head from h to the draft logits (and normalisers). */
+sv_status spec_verify_lowrank_head(const void* h, const void* w_down, const void* w_up, int M, int d, int r,
+                                   int V, const float* temperature, void* out_logits, double* out_lse,
+                                   void* workspace, size_t workspace_bytes, int32_t* out_error,
+                                   struct CUstream_st* stream);
+
 #ifdef __cplusplus
 }
 #endif

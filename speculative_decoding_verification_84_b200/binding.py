@@ -23,7 +23,9 @@ EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_
             "spec_verify_status_string", "spec_verify_kernels_per_call", "spec_verify_noalloc",
             "spec_verify_fanout", "spec_verify_topf", "spec_verify_cache_lookup",
             "spec_verify_bandit_state_size", "spec_verify_bandit_init", "spec_verify_bandit_step",
-            "spec_verify_bandit_simulate", "spec_verify_tree", "spec_verify_tree_prune")
+            "spec_verify_bandit_simulate", "spec_verify_tree", "spec_verify_tree_prune",
+            "spec_verify_lowrank_workspace_size", "spec_verify_lowrank_down", "spec_verify_lowrank_up",
+            "spec_verify_lowrank_head")
 MAX_TOPF = 32
 MAX_ARMS = 16
 BANDIT_UCB1, BANDIT_THOMPSON = 0, 1
@@ -78,6 +80,14 @@ def load_library(path: str = LIB_PATH):
     lib.spec_verify_tree.restype = i32
     lib.spec_verify_tree_prune.argtypes = [vp, i32, vp, vp, vp, ctypes.c_double, i32, i32, i32, vp, vp, vp]
     lib.spec_verify_tree_prune.restype = i32
+    lib.spec_verify_lowrank_workspace_size.argtypes = [i32, i32, i32]
+    lib.spec_verify_lowrank_workspace_size.restype = sz
+    lib.spec_verify_lowrank_down.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
+    lib.spec_verify_lowrank_down.restype = i32
+    lib.spec_verify_lowrank_up.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp]
+    lib.spec_verify_lowrank_up.restype = i32
+    lib.spec_verify_lowrank_head.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp]
+    lib.spec_verify_lowrank_head.restype = i32
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -386,6 +396,85 @@ def tree_prune(draft: torch.Tensor, parent: torch.Tensor, tokens: torch.Tensor, 
                                              temperature.data_ptr(), float(threshold), B, N, V, keep.data_ptr(),
                                              cum.data_ptr(), s.cuda_stream))
     return keep, cum
+
+
+def _bf16_2d(t, name, shape, device):
+    _check(t, name, torch.bfloat16, shape, device)
+
+
+def lowrank_down(h: torch.Tensor, w_down: torch.Tensor, *, error: torch.Tensor | None = None,
+                 stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """u = bf16(h W_down^T) on the tensor cores: h [M, d], W_down [r, d] bf16 -> [M, r]."""
+    lib = load_library()
+    device = h.device
+    M, d = h.shape
+    r = w_down.shape[0]
+    _bf16_2d(h, "h", (M, d), device)
+    _bf16_2d(w_down, "w_down", (r, d), device)
+    u = torch.empty((M, r), dtype=torch.bfloat16, device=device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_lowrank_down(h.data_ptr(), w_down.data_ptr(), M, d, r, u.data_ptr(),
+                                               error.data_ptr() if error is not None else None, s.cuda_stream))
+    return u
+
+
+def lowrank_up(u: torch.Tensor, w_up: torch.Tensor, temperature: torch.Tensor | None = None, *,
+               with_lse: bool = True, error: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """z = bf16(u W_up^T) [M, V] and (with_lse) each row's log-normaliser at its temperature."""
+    lib = load_library()
+    device = u.device
+    M, r = u.shape
+    V = w_up.shape[0]
+    _bf16_2d(u, "u", (M, r), device)
+    _bf16_2d(w_up, "w_up", (V, r), device)
+    if temperature is not None:
+        _check(temperature, "temperature", torch.float32, (M,), device)
+    z = torch.empty((M, V), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((M,), dtype=torch.float64, device=device) if with_lse else None
+    ws = torch.empty(lib.spec_verify_lowrank_workspace_size(M, r, V), dtype=torch.uint8, device=device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_lowrank_up(u.data_ptr(), w_up.data_ptr(), M, r, V,
+                                             temperature.data_ptr() if temperature is not None else None,
+                                             z.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                             ws.data_ptr(), ws.numel(), error.data_ptr() if error is not None else None,
+                                             s.cuda_stream))
+    return (z, lse) if with_lse else z
+
+
+def lowrank_head(h: torch.Tensor, w_down: torch.Tensor, w_up: torch.Tensor, temperature: torch.Tensor | None = None,
+                 *, error: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                 stream: torch.cuda.Stream | None = None):
+    """The low-rank draft head: (z [M, V] bf16 logits, lse [M] float64)."""
+    lib = load_library()
+    device = h.device
+    M, d = h.shape
+    r = w_down.shape[0]
+    V = w_up.shape[0]
+    _bf16_2d(h, "h", (M, d), device)
+    _bf16_2d(w_down, "w_down", (r, d), device)
+    _bf16_2d(w_up, "w_up", (V, r), device)
+    if temperature is not None:
+        _check(temperature, "temperature", torch.float32, (M,), device)
+    z = torch.empty((M, V), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((M,), dtype=torch.float64, device=device)
+    if workspace is None:
+        workspace = torch.empty(lib.spec_verify_lowrank_workspace_size(M, r, V), dtype=torch.uint8, device=device)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        _raise_if(lib.spec_verify_lowrank_head(h.data_ptr(), w_down.data_ptr(), w_up.data_ptr(), M, d, r, V,
+                                               temperature.data_ptr() if temperature is not None else None,
+                                               z.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                               error.data_ptr() if error is not None else None, s.cuda_stream))
+    return z, lse
+
+
+def lowrank_to_device(w, device="cuda"):
+    """Copy a ``workloads.LowRankWorkload`` to torch tensors on ``device``."""
+    def bf(a):
+        return torch.from_numpy(a).view(torch.bfloat16).to(device)
+    return dict(h=bf(w.h), w_down=bf(w.w_down), w_up=bf(w.w_up), temperature=torch.from_numpy(w.temperature).to(device))
 
 
 def tree_to_device(w, device="cuda"):

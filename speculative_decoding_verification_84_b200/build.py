@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "spec_verify.cu")
 DEPS = [os.path.join(HERE, "csrc", f)
         for f in ("sv_common.cuh", "sv_generic.cuh", "sv_pass.cuh", "sv_small.cuh", "sv_topf.cuh", "sv_bandit.cuh",
-                  "sv_tree.cuh")]
+                  "sv_tree.cuh", "sv_lowrank.cuh")]
 HEADER = os.path.join(ROOT, "include", "spec_verify.h")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libspecverify.so")

@@ -32,6 +32,7 @@
 #include "sv_topf.cuh"
 #include "sv_bandit.cuh"
 #include "sv_tree.cuh"
+#include "sv_lowrank.cuh"
 
 namespace {
 
@@ -784,4 +785,146 @@ extern "C" sv_status spec_verify_tree_prune(const void* draft_logits, sv_dtype d
     if (cudaGetLastError() != cudaSuccess) return SV_ERR_CUDA;
     sv::sv_tree_prune_walk<<<(unsigned)cdiv(B, 128), 128, 0, st>>>(g);
     return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------- low-rank draft head
+
+namespace {
+
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+TensorMapEncodeFn tensor_map_encoder()
+{
+    static TensorMapEncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<TensorMapEncodeFn>(f);
+    });
+    return fn;
+}
+
+// Tensor map of a row-major [rows][K] bf16 matrix, loaded as boxes of 64 (K) x
+// box_rows with the 128-byte swizzle; out-of-range elements read as zero.
+bool lr_map(CUtensorMap* m, const void* base, long long rows, long long K, int box_rows)
+{
+    TensorMapEncodeFn enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)sv::kLrBK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t lr_launch(const void* A, const void* B, int M, int N, int K, void* out, float4* part,
+                      const float* temperature, int* err, cudaStream_t st)
+{
+    CUtensorMap ta, tb;
+    if (!lr_map(&ta, A, M, K, sv::kLrBM) || !lr_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
+    constexpr int smem = sv::lr_smem_bytes<BN>();
+    static std::once_flag once[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaError_t attr_err = cudaSuccess;
+    if (dev >= 0 && dev < kMaxDevices)
+        std::call_once(once[dev], [&] {
+            attr_err = cudaFuncSetAttribute(sv::sv_lr_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        });
+    if (attr_err != cudaSuccess) return attr_err;
+    sv::LrArgs g;
+    g.out = static_cast<__nv_bfloat16*>(out);
+    g.part = part;
+    g.temperature = temperature;
+    g.err = err;
+    g.M = M; g.N = N; g.K = K;
+    g.m_tiles = (int)cdiv(M, sv::kLrBM);
+    g.n_tiles = (int)cdiv(N, BN);
+    const long long grid = (long long)g.m_tiles * g.n_tiles;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    sv::sv_lr_gemm<BN><<<(unsigned)grid, sv::kLrThreads, smem, st>>>(ta, tb, g);
+    return cudaGetLastError();
+}
+
+bool lr_shape_ok(int M, int d, int r, int V)
+{
+    // K a multiple of 8: the tensor maps' row pitch must be a multiple of 16 bytes
+    return M >= 1 && d >= 8 && r >= 8 && V >= 1 && (d % 8) == 0 && (r % 8) == 0 && V <= SV_MAX_V &&
+           (long long)M * r < (1LL << 40);
+}
+
+constexpr int kLrUpBN = 256;
+constexpr int kLrDownBN = 32;
+
+size_t lr_u_bytes(int M, int r) { return ((size_t)M * r * 2 + 1023) / 1024 * 1024; }
+size_t lr_part_bytes(int M, int V) { return (size_t)M * (size_t)cdiv(V, kLrUpBN) * sizeof(float4); }
+
+}  // namespace
+
+extern "C" size_t spec_verify_lowrank_workspace_size(int M, int r, int V)
+{
+    if (M < 1 || r < 8 || (r % 8) != 0 || V < 1 || V > SV_MAX_V) return 0;
+    return lr_u_bytes(M, r) + lr_part_bytes(M, V);
+}
+
+extern "C" sv_status spec_verify_lowrank_down(const void* h, const void* w_down, int M, int d, int r, void* out_u,
+                                              int32_t* out_error, struct CUstream_st* stream)
+{
+    if (!h || !w_down || !out_u || !lr_shape_ok(M, d, r, 1)) return SV_ERR_INVALID_ARG;
+    if (!aligned(h, 16) || !aligned(w_down, 16) || !aligned(out_u, 16) || !aligned(out_error, 4))
+        return SV_ERR_MISALIGNED;
+    const cudaError_t e = lr_launch<kLrDownBN>(h, w_down, M, r, d, out_u, nullptr, nullptr, out_error,
+                                               (cudaStream_t)stream);
+    return e == cudaSuccess ? SV_OK : (e == cudaErrorInvalidValue ? SV_ERR_INVALID_ARG : SV_ERR_CUDA);
+}
+
+extern "C" sv_status spec_verify_lowrank_up(const void* u, const void* w_up, int M, int r, int V,
+                                            const float* temperature, void* out_logits, double* out_lse,
+                                            void* workspace, size_t workspace_bytes, int32_t* out_error,
+                                            struct CUstream_st* stream)
+{
+    if (!u || !w_up || !out_logits || !lr_shape_ok(M, 8, r, V)) return SV_ERR_INVALID_ARG;
+    if (!aligned(u, 16) || !aligned(w_up, 16) || !aligned(out_logits, 16) || !aligned(temperature, 4) ||
+        !aligned(out_lse, 8) || !aligned(out_error, 4) || !aligned(workspace, 256))
+        return SV_ERR_MISALIGNED;
+    float4* part = nullptr;
+    if (out_lse) {
+        if (!workspace || workspace_bytes < lr_part_bytes(M, V)) return SV_ERR_WORKSPACE_TOO_SMALL;
+        part = static_cast<float4*>(workspace);
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = lr_launch<kLrUpBN>(u, w_up, M, V, r, out_logits, part, temperature, out_error, st);
+    if (e != cudaSuccess) return e == cudaErrorInvalidValue ? SV_ERR_INVALID_ARG : SV_ERR_CUDA;
+    if (out_lse) {
+        sv::sv_lr_lse<<<(unsigned)cdiv((long long)M * 32, 256), 256, 0, st>>>(part, temperature, M,
+                                                                            (int)cdiv(V, kLrUpBN), out_lse);
+        if (cudaGetLastError() != cudaSuccess) return SV_ERR_CUDA;
+    }
+    return SV_OK;
+}
+
+extern "C" sv_status spec_verify_lowrank_head(const void* h, const void* w_down, const void* w_up, int M, int d,
+                                              int r, int V, const float* temperature, void* out_logits,
+                                              double* out_lse, void* workspace, size_t workspace_bytes,
+                                              int32_t* out_error, struct CUstream_st* stream)
+{
+    if (!h || !w_down || !w_up || !out_logits || !lr_shape_ok(M, d, r, V)) return SV_ERR_INVALID_ARG;
+    if (!workspace) return SV_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return SV_ERR_MISALIGNED;
+    if (workspace_bytes < spec_verify_lowrank_workspace_size(M, r, V)) return SV_ERR_WORKSPACE_TOO_SMALL;
+    void* u = workspace;
+    void* rest = static_cast<unsigned char*>(workspace) + lr_u_bytes(M, r);
+    const sv_status s = spec_verify_lowrank_down(h, w_down, M, d, r, u, out_error, stream);
+    if (s != SV_OK) return s;
+    return spec_verify_lowrank_up(u, w_up, M, r, V, temperature, out_logits, out_lse, rest,
+                                  workspace_bytes - lr_u_bytes(M, r), out_error, stream);
 }

@@ -1,0 +1,338 @@
+// sv_lowrank.cuh -- the low-rank draft head on the 5th-generation tensor cores
+// [SlimSpec, Metodologia, "Arquitetura": z = W_up W_down h, W_down in R^{r x d},
+// W_up in R^{V x r}, r << d, in place of the full-rank z = W_full h].
+//
+// Both contractions are out = A B^T with A [rows][K] and B [cols][K] bf16,
+// K-major (the layout of h, W_down and W_up as stored), fp32 accumulation:
+//   down:  u [M][r] = h [M][d]  W_down [r][d]^T   (rounded to bf16: the second
+//          contraction takes bf16 operands)
+//   up:    z [M][V] = u [M][r]  W_up [V][r]^T     (bf16 logits for the verifier)
+// and the up contraction's epilogue also folds each row's online log-sum-exp of
+// its bf16 logits at the row's temperature (the draft row's normaliser, the
+// arithmetic of the verifier's passes), written as one partial per (row,
+// column tile) and folded by sv_lr_lse.
+//
+// sv_lr_gemm: one CTA per 128 x BN output tile (column tiles outer, so the
+// row tiles sharing a W tile run together and read it once from HBM).
+//   warp 0 (one thread)  TMA: 128 x 64 of A and BN x 64 of B per stage, 128-byte
+//                        swizzle, kLrStages stages, mbarrier transaction counts
+//   warp 1 (one thread)  tcgen05.mma kind::f16 (bf16 x bf16 -> f32), M = 128,
+//                        N = BN, four K = 16 steps per stage, accumulator in
+//                        TMEM; tcgen05.commit frees the stage, and after the last
+//                        stage signals the epilogue
+//   warp 2               allocates and frees the TMEM columns
+//   warps 4-7            epilogue: tcgen05.ld of 32 lanes x 32 columns at a
+//                        time (warp 4 + q reads lanes 32q..32q+31), bf16 rounding,
+//                        16-byte stores, the row's online log-sum-exp
+// Every wait on an mbarrier is bounded: past kLrSpin polls the CTA raises
+// *err, stops issuing, and still frees its TMEM.
+#pragma once
+
+#include <cuda.h>  // CUtensorMap
+#include <cuda_bf16.h>
+
+#include "sv_common.cuh"
+
+namespace sv {
+
+constexpr int kLrBM = 128;      // tile rows = the MMA's M
+constexpr int kLrBK = 64;       // K per stage: one 128-byte swizzled row of bf16
+constexpr int kLrStages = 4;
+constexpr int kLrThreads = 256;
+constexpr unsigned kLrSpin = 1u << 24;
+
+struct LrArgs {
+    __nv_bfloat16* out;        // [M][N]
+    float4* part;              // [M][n_tiles] (m, mk, s, 0) or null (no normaliser)
+    const float* temperature;  // [M] or null (T = 1)
+    int* err;                  // optional: 1 if a wait gave up
+    int M, N, K;
+    int m_tiles, n_tiles;
+};
+
+__device__ __forceinline__ uint32_t lr_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void lr_mbar_init(uint64_t* bar, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(lr_smem(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void lr_expect_tx(uint64_t* bar, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(lr_smem(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool lr_try_wait(uint64_t* bar, unsigned parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(lr_smem(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with this parity; false (after raising the flags) if it did
+// not complete within kLrSpin polls, or another role of the CTA already gave up.
+__device__ __forceinline__ bool lr_wait(uint64_t* bar, unsigned parity, volatile int* abort, int* err)
+{
+    for (unsigned i = 0; i < kLrSpin; ++i) {
+        if (lr_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && *abort) return false;
+    }
+    *abort = 1;
+    if (err) atomicExch(err, 1);
+    return false;
+}
+
+__device__ __forceinline__ void lr_tma_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            lr_smem(dst)),
+        "l"((uint64_t)map), "r"(lr_smem(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t lr_desc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu)   // start address, 16-byte units
+           | ((uint64_t)1 << 16)                 // leading byte offset (unused for swizzled K-major)
+           | ((uint64_t)(1024 >> 4) << 32)       // stride byte offset: 8 rows x 128 bytes
+           | ((uint64_t)1 << 46)                 // descriptor version (sm_100)
+           | ((uint64_t)2 << 61);                // layout: 128-byte swizzle
+}
+
+// Instruction descriptor: f32 accumulator, bf16 A and B, both K-major, M x N.
+template <int N>
+__device__ __forceinline__ constexpr uint32_t lr_idesc()
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kLrBM >> 4) << 24);
+}
+
+__device__ __forceinline__ void lr_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
+__device__ __forceinline__ void lr_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(lr_smem(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void lr_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void lr_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void lr_tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int BN>
+constexpr int lr_smem_bytes()
+{
+    return kLrStages * (kLrBM * kLrBK * 2 + BN * kLrBK * 2) + 1024;  // + alignment slack
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kLrThreads, 1)
+    sv_lr_gemm(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, LrArgs g)
+{
+    static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "tile columns: a power of two TMEM allocation");
+    constexpr int A_BYTES = kLrBM * kLrBK * 2;
+    constexpr int B_BYTES = BN * kLrBK * 2;
+    constexpr int STAGE = A_BYTES + B_BYTES;
+    extern __shared__ unsigned char lr_dyn[];
+    // the stages start on a 1024-byte boundary of the shared window (the swizzle atom)
+    unsigned char* sm = lr_dyn + ((1024u - (lr_smem(lr_dyn) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t full[kLrStages], empty[kLrStages], done;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort, s_consumed;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m_tile = (int)(blockIdx.x % (unsigned)g.m_tiles), n_tile = (int)(blockIdx.x / (unsigned)g.m_tiles);
+    const int kbs = (g.K + kLrBK - 1) / kLrBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kLrStages; ++s) {
+            lr_mbar_init(&full[s], 1);
+            lr_mbar_init(&empty[s], 1);
+        }
+        lr_mbar_init(&done, 1);
+        s_abort = 0;
+        s_consumed = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(lr_smem(&s_tmem)),
+                     "r"((uint32_t)BN));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    lr_fence_before();
+    __syncthreads();
+    lr_fence_after();
+    const uint32_t tmem = s_tmem;
+    volatile int* abort = &s_abort;
+
+    int issued = 0;
+    if (warp == 0 && lane == 0) {
+        // ---- producer
+        for (int kb = 0; kb < kbs; ++kb) {
+            const int s = kb % kLrStages;
+            const unsigned round = (unsigned)(kb / kLrStages);
+            if (kb >= kLrStages && !lr_wait(&empty[s], (round - 1u) & 1u, abort, g.err)) break;
+            unsigned char* st = sm + s * STAGE;
+            lr_expect_tx(&full[s], (unsigned)STAGE);
+            lr_tma_2d(st, &ta, &full[s], kb * kLrBK, m_tile * kLrBM);
+            lr_tma_2d(st + A_BYTES, &tb, &full[s], kb * kLrBK, n_tile * BN);
+            issued = kb + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer
+        constexpr uint32_t idesc = lr_idesc<BN>();
+        for (int kb = 0; kb < kbs; ++kb) {
+            const int s = kb % kLrStages;
+            const unsigned round = (unsigned)(kb / kLrStages);
+            if (!lr_wait(&full[s], round & 1u, abort, g.err)) break;
+            lr_fence_after();
+            const uint32_t a0 = lr_smem(sm + s * STAGE), b0 = a0 + A_BYTES;
+#pragma unroll
+            for (int j = 0; j < kLrBK / 16; ++j)  // K = 16 per MMA: 32 bytes along the swizzled row
+                lr_mma(tmem, lr_desc(a0 + 32 * j), lr_desc(b0 + 32 * j), idesc, (kb > 0 || j > 0) ? 1u : 0u);
+            lr_commit(&empty[s]);
+            s_consumed = kb + 1;
+        }
+        lr_commit(&done);
+    } else if (warp >= 4) {
+        // ---- epilogue: warp 4 + q owns TMEM lanes (= tile rows) 32q .. 32q + 31
+        const int q = warp - 4;
+        const int row = m_tile * kLrBM + 32 * q + lane;
+        const bool row_ok = row < g.M;
+        const bool lse = g.part != nullptr;
+        float T = 1.f;
+        if (lse && g.temperature && row_ok) T = g.temperature[row];
+        const bool lse_row = lse && row_ok && T > 0.f && T <= FLT_MAX;
+        float khi = 0.f, klo = 0.f;
+        if (lse_row) split_k(T, &khi, &klo);
+        Lse L;
+        lse_init(L);
+        // one lane waits, so the warp-wide tcgen05.ld below runs on all lanes or none
+        int ready = 0;
+        if (lane == 0) ready = lr_wait(&done, 0u, abort, g.err) ? 1 : 0;
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (ready) {
+            lr_fence_after();
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t r[32];
+                lr_tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, r);
+                const int n0 = n_tile * BN + c;
+                float x[32];
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                    packed[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                    x[i] = __bfloat162float(h2.x);
+                    x[i + 1] = __bfloat162float(h2.y);
+                }
+                if (row_ok) {
+                    __nv_bfloat16* dst = g.out + (size_t)row * g.N + n0;
+                    if (n0 + 32 <= g.N && (g.N & 7) == 0) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            reinterpret_cast<uint4*>(dst)[v] =
+                                make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    } else {
+                        for (int i = 0; i < 32 && n0 + i < g.N; ++i) {
+                            const uint32_t w = packed[i / 2];
+                            const unsigned short hb = (unsigned short)((i & 1) ? (w >> 16) : (w & 0xffffu));
+                            reinterpret_cast<unsigned short*>(dst)[i] = hb;
+                        }
+                    }
+                }
+                if (lse_row) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (n0 + i >= g.N) x[i] = -INFINITY;  // columns past N take no part
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) lse_add<8>(L, x + i, khi, klo);
+                }
+            }
+        }
+        if (lse && row_ok) g.part[(size_t)row * g.n_tiles + n_tile] = make_float4(L.m, L.mk, L.s, 0.f);
+    }
+    lr_fence_before();
+    __syncthreads();
+    // after a wait gave up: let the copies this CTA issued but never consumed land
+    // (bounded) before its shared memory goes away
+    if (warp == 0 && lane == 0 && s_abort)
+        for (int kb = s_consumed; kb < issued; ++kb) {
+            const unsigned par = (unsigned)(kb / kLrStages) & 1u;
+            for (unsigned i = 0; i < kLrSpin && !lr_try_wait(&full[kb % kLrStages], par); ++i) {
+            }
+        }
+    if (warp == 2) {
+        lr_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)BN));
+    }
+}
+
+// One warp per row: fold the row's column-tile partials into lse = (MK + log2 S) ln 2
+// (NaN for T = 0, an invalid T, or a row with NaN or +inf).
+__global__ void sv_lr_lse(const float4* __restrict__ part, const float* __restrict__ temperature, int M, int n_tiles,
+                          double* __restrict__ out_lse)
+{
+    const int row = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (row >= M) return;
+    const float T = temperature ? temperature[row] : 1.f;
+    float M_ = -INFINITY, MK = 0.f;
+    double S = 0.0;
+    int nan = 0;
+    for (int t = lane; t < n_tiles; t += 32) {
+        const float4 p = part[(size_t)row * n_tiles + t];
+        nan |= (p.z != p.z);
+        if (p.x == -INFINITY) continue;
+        if (M_ == -INFINITY) { M_ = p.x; MK = p.y; S = (double)p.z; continue; }
+        if (p.y > MK) { S = S * pow2d(MK - p.y) + (double)p.z; MK = p.y; }
+        else S += (double)p.z * pow2d(p.y - MK);
+        M_ = fmaxf(M_, p.x);
+    }
+    // fold the lanes (xor tree: every lane ends with the same values)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, M_, o);
+        const float mk2 = __shfl_xor_sync(0xffffffffu, MK, o);
+        const double s2 = __shfl_xor_sync(0xffffffffu, S, o);
+        nan |= __shfl_xor_sync(0xffffffffu, nan, o);
+        if (m2 == -INFINITY) continue;
+        if (M_ == -INFINITY) { M_ = m2; MK = mk2; S = s2; continue; }
+        if (mk2 > MK) { S = S * pow2d(MK - mk2) + s2; MK = mk2; }
+        else S += s2 * pow2d(mk2 - MK);
+        M_ = fmaxf(M_, m2);
+    }
+    if (lane == 0) {
+        const bool ok = T > 0.f && T <= FLT_MAX && !nan && M_ != -INFINITY && M_ != INFINITY && S > 0.0 && S <= DBL_MAX;
+        out_lse[row] = ok ? ((double)MK + log2(S)) * kLn2 : (double)NAN;
+    }
+}
+
+}  // namespace sv
