@@ -41,6 +41,7 @@ WORKLOAD = "c3"
 WORKLOAD_DESC = ("spec_verify B=64, gamma=5, V=128256, bf16 logits; target N(0,3^2)+Zipf(1.1) log-bias, "
                  "draft rho=0.9, T=1.0 (synthetic, seed 86)")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def algorithmic_bytes(B, gamma, V, esz):
@@ -49,6 +50,17 @@ def algorithmic_bytes(B, gamma, V, esz):
     small_in = (gamma + gamma + 1 + 1) * 4 * B          # tokens, u_accept, u_resample, T
     outs = (gamma + 1 + 1) * 4 * B                      # out_tokens, n_accepted
     return logits + small_in + outs
+
+
+def tc_peak():
+    """Dense bf16 tensor throughput (TFLOP/s) for a kernel timed alone: the measured
+    burst figure, else the pool's earlier measurement (1590)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def peaks():
@@ -509,6 +521,76 @@ def tree_row_line(dev, lib, binding, peak, peak_kind, cpu_seconds=2.0):
                              "sample": f"{reps} passes over the 64 trees"}}
 
 
+LOWRANK_SHAPE = (320, 4096, 512, 128256)  # M = 64 sequences x gamma 5, d, r = d/8, V
+
+
+def lowrank_row_line(dev, lib, binding, peak, peak_kind):
+    """The low-rank draft head (SlimSpec) on M = 320 draft positions (the c3 batch:
+    64 sequences x gamma 5), d = 4096, r = d/8 = 512, V = 128256: the two tcgen05
+    contractions and the whole head, each timed as CUDA graph replays over 3
+    copies of W_up (394 MB > 2x L2).  Algorithmic bytes: both operands read once
+    and the output written once; FLOPs 2 M N K.  The up contraction is bound by
+    HBM (its time at the HBM peak is above its time at the tensor peak)."""
+    import torch
+    from speculative_decoding_verification_84_b200 import workloads as W
+    M, d, r, V = LOWRANK_SHAPE
+    w = W.make_lowrank(M, d, r, V, seed=2005, T=1.0)
+    base = binding.lowrank_to_device(w, dev)
+    n_copies = 3
+    w_ups = [base["w_up"]] + [base["w_up"].clone() for _ in range(n_copies - 1)]
+    z = torch.empty((M, V), dtype=torch.bfloat16, device=dev)
+    u = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((M,), dtype=torch.float64, device=dev)
+    ws = torch.empty(lib.spec_verify_lowrank_workspace_size(M, r, V), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    T = base["temperature"]
+
+    def head(i):
+        rc = lib.spec_verify_lowrank_head(base["h"].data_ptr(), base["w_down"].data_ptr(), w_ups[i % n_copies].data_ptr(),
+                                          M, d, r, V, T.data_ptr(), z.data_ptr(), lse.data_ptr(), ws.data_ptr(),
+                                          ws.numel(), err.data_ptr(), stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(binding.status_string(rc))
+
+    def down(i):
+        rc = lib.spec_verify_lowrank_down(base["h"].data_ptr(), base["w_down"].data_ptr(), M, d, r, u.data_ptr(),
+                                          err.data_ptr(), stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(binding.status_string(rc))
+
+    def up(i):
+        rc = lib.spec_verify_lowrank_up(u.data_ptr(), w_ups[i % n_copies].data_ptr(), M, r, V, T.data_ptr(),
+                                        z.data_ptr(), lse.data_ptr(), ws.data_ptr(), ws.numel(), err.data_ptr(),
+                                        stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(binding.status_string(rc))
+
+    with torch.cuda.stream(stream):
+        for i in range(4):
+            head(i)
+    torch.cuda.synchronize()
+    ms_head = graph_ms(stream, head, 300, n_copies)
+    ms_down = graph_ms(stream, down, 300, n_copies)
+    ms_up = graph_ms(stream, up, 300, n_copies)
+    tc, tc_kind = tc_peak()
+    alg_up = V * r * 2 + M * r * 2 + M * V * 2
+    fl_up = 2.0 * M * V * r
+    alg_down = M * d * 2 + r * d * 2 + M * r * 2
+    fl_down = 2.0 * M * r * d
+    t_up_bound = max(alg_up / (peak * 1e9), fl_up / (tc * 1e12))
+    return {"workload": "h3: M=320 (64 sequences x gamma 5), d=4096, r=512, V=128256, bf16 weights random-init",
+            "us_per_call_head": 1e3 * ms_head, "us_per_call_down": 1e3 * ms_down, "us_per_call_up": 1e3 * ms_up,
+            "up": {"algorithmic_bytes": alg_up, "flops": fl_up, "hbm_gbs": alg_up / (ms_up / 1e3) / 1e9,
+                   "tflops": fl_up / (ms_up / 1e3) / 1e12, "frac_of_hbm_peak": alg_up / (ms_up / 1e3) / 1e9 / peak,
+                   "frac_of_tensor_peak": fl_up / (ms_up / 1e3) / 1e12 / tc, "bound": "hbm",
+                   "frac_of_roofline": t_up_bound / (ms_up / 1e3)},
+            "down": {"algorithmic_bytes": alg_down, "flops": fl_down, "tflops": fl_down / (ms_down / 1e3) / 1e12},
+            "peak_hbm_gbs": peak, "peak_source": peak_kind, "peak_bf16_tflops": tc, "tensor_peak_source": tc_kind,
+            "error_flag": int(err.item()),
+            "l2": f"{n_copies} copies of W_up rotated ({n_copies * V * r * 2 / 1e6:.0f} MB)"}
+
+
 def cache_row_line(w, dev, lib, binding, peak, peak_kind, budget_ms=20.0):
     """The speculation-cache row on one workload: spec_verify_topf with the
     geometric fan-out of a 64-slot budget at acceptance rate 0.7 (then at most 32
@@ -698,6 +780,8 @@ def run_ours(args):
         torch.cuda.empty_cache()
         per_config["tree_row_t3"] = tree_row_line(dev, lib, binding, peak, peak_kind)
         torch.cuda.empty_cache()
+        per_config["lowrank_head_h3"] = lowrank_row_line(dev, lib, binding, peak, peak_kind)
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -761,6 +845,15 @@ def run_profile(args):
     from speculative_decoding_verification_84_b200 import binding, build, workloads as W
     build.build()
     lib = binding.load_library()
+    if args.profile == "h3":
+        M, d, r, V = LOWRANK_SHAPE
+        w = W.make_lowrank(M, d, r, V, seed=2005, T=1.0)
+        dv = binding.lowrank_to_device(w, "cuda:0")
+        for i in range(args.warmup + args.steps):
+            binding.lowrank_head(dv["h"], dv["w_down"], dv["w_up"], dv["temperature"])
+        torch.cuda.synchronize()
+        print(f"h3: {args.warmup + args.steps} calls, 3 launches each", flush=True)
+        return 0
     if args.profile == "t3":
         w = W.make_tree(64, TREE_SHAPE, 128256, "bf16", seed=91, name="t3")
         d = binding.tree_to_device(w, "cuda:0")
@@ -787,7 +880,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="skip the line's per-workload numbers")
-    ap.add_argument("--profile", choices=list(PER_CONFIG) + ["t3"], default=None,
+    ap.add_argument("--profile", choices=list(PER_CONFIG) + ["t3", "h3"], default=None,
                     help="only make warm-up + K calls of this workload (for a profiler); no JSON line")
     args = ap.parse_args()
     if args.profile:

@@ -849,8 +849,9 @@ cudaError_t lr_launch(const void* A, const void* B, int M, int N, int K, void* o
     g.M = M; g.N = N; g.K = K;
     g.m_tiles = (int)cdiv(M, sv::kLrBM);
     g.n_tiles = (int)cdiv(N, BN);
-    const long long grid = (long long)g.m_tiles * g.n_tiles;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const long long tiles = (long long)g.m_tiles * g.n_tiles;
+    if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const long long grid = std::min<long long>(tiles, device_sm_count());  // one CTA per SM (shared memory)
     sv::sv_lr_gemm<BN><<<(unsigned)grid, sv::kLrThreads, smem, st>>>(ta, tb, g);
     return cudaGetLastError();
 }
@@ -866,7 +867,7 @@ constexpr int kLrUpBN = 256;
 constexpr int kLrDownBN = 32;
 
 size_t lr_u_bytes(int M, int r) { return ((size_t)M * r * 2 + 1023) / 1024 * 1024; }
-size_t lr_part_bytes(int M, int V) { return (size_t)M * (size_t)cdiv(V, kLrUpBN) * sizeof(float4); }
+size_t lr_part_bytes(int M, int V) { return (size_t)M * (size_t)cdiv(V, kLrUpBN) * 2 * sizeof(float4); }
 
 }  // namespace
 
@@ -906,7 +907,7 @@ extern "C" sv_status spec_verify_lowrank_up(const void* u, const void* w_up, int
     if (e != cudaSuccess) return e == cudaErrorInvalidValue ? SV_ERR_INVALID_ARG : SV_ERR_CUDA;
     if (out_lse) {
         sv::sv_lr_lse<<<(unsigned)cdiv((long long)M * 32, 256), 256, 0, st>>>(part, temperature, M,
-                                                                            (int)cdiv(V, kLrUpBN), out_lse);
+                                                                            2 * (int)cdiv(V, kLrUpBN), out_lse);
         if (cudaGetLastError() != cudaSuccess) return SV_ERR_CUDA;
     }
     return SV_OK;

@@ -12,8 +12,9 @@
 // arithmetic of the verifier's passes), written as one partial per (row,
 // column tile) and folded by sv_lr_lse.
 //
-// sv_lr_gemm: one CTA per 128 x BN output tile (column tiles outer, so the
-// row tiles sharing a W tile run together and read it once from HBM).
+// sv_lr_gemm: persistent, one CTA per SM walking 128 x BN output tiles (column
+// tiles outer, so the row tiles sharing a W tile run together and read it once
+// from HBM), the accumulator double-buffered in TMEM.
 //   warp 0 (one thread)  TMA: 128 x 64 of A and BN x 64 of B per stage, 128-byte
 //                        swizzle, kLrStages stages, mbarrier transaction counts
 //   warp 1 (one thread)  tcgen05.mma kind::f16 (bf16 x bf16 -> f32), M = 128,
@@ -21,9 +22,10 @@
 //                        TMEM; tcgen05.commit frees the stage, and after the last
 //                        stage signals the epilogue
 //   warp 2               allocates and frees the TMEM columns
-//   warps 4-7            epilogue: tcgen05.ld of 32 lanes x 32 columns at a
-//                        time (warp 4 + q reads lanes 32q..32q+31), bf16 rounding,
-//                        16-byte stores, the row's online log-sum-exp
+//   warps 4-11           epilogue: tcgen05.ld of 32 lanes x 32 columns at a
+//                        time (warp 4 + w reads lanes 32 (w % 4) ... + 31 and
+//                        columns half w / 4), bf16 rounding, 16-byte stores, the
+//                        row's online log-sum-exp over its half of the columns
 // Every wait on an mbarrier is bounded: past kLrSpin polls the CTA raises
 // *err, stops issuing, and still frees its TMEM.
 #pragma once
@@ -38,12 +40,13 @@ namespace sv {
 constexpr int kLrBM = 128;      // tile rows = the MMA's M
 constexpr int kLrBK = 64;       // K per stage: one 128-byte swizzled row of bf16
 constexpr int kLrStages = 4;
-constexpr int kLrThreads = 256;
+constexpr int kLrEpiWarps = 8;  // two per TMEM lane quarter, each on half the columns
+constexpr int kLrThreads = 128 + 32 * kLrEpiWarps;
 constexpr unsigned kLrSpin = 1u << 24;
 
 struct LrArgs {
     __nv_bfloat16* out;        // [M][N]
-    float4* part;              // [M][n_tiles] (m, mk, s, 0) or null (no normaliser)
+    float4* part;              // [M][2 n_tiles] (m, mk, s, 0) per column half, or null
     const float* temperature;  // [M] or null (T = 1)
     int* err;                  // optional: 1 if a wait gave up
     int M, N, K;
@@ -153,6 +156,16 @@ constexpr int lr_smem_bytes()
     return kLrStages * (kLrBM * kLrBK * 2 + BN * kLrBK * 2) + 1024;  // + alignment slack
 }
 
+__device__ __forceinline__ void lr_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(lr_smem(bar)) : "memory");
+}
+
+// Persistent: CTA c takes tiles c, c + gridDim.x, ... (consecutive tiles share a
+// column tile, so the row tiles of one W tile run at the same time).  The
+// accumulator is double-buffered in TMEM (2 x BN columns): while the epilogue
+// warps drain tile i from one buffer, the MMA thread fills the other with tile
+// i + 1, and the producer keeps loading ahead through the stage ring.
 template <int BN>
 __global__ void __launch_bounds__(kLrThreads, 1)
     sv_lr_gemm(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, LrArgs g)
@@ -161,30 +174,34 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     constexpr int A_BYTES = kLrBM * kLrBK * 2;
     constexpr int B_BYTES = BN * kLrBK * 2;
     constexpr int STAGE = A_BYTES + B_BYTES;
+    constexpr uint32_t kCols = 2 * BN;  // two accumulators
     extern __shared__ unsigned char lr_dyn[];
     // the stages start on a 1024-byte boundary of the shared window (the swizzle atom)
     unsigned char* sm = lr_dyn + ((1024u - (lr_smem(lr_dyn) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t full[kLrStages], empty[kLrStages], done;
+    __shared__ __align__(8) uint64_t full[kLrStages], empty[kLrStages], tfull[2], tempty[2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort, s_consumed;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m_tile = (int)(blockIdx.x % (unsigned)g.m_tiles), n_tile = (int)(blockIdx.x / (unsigned)g.m_tiles);
     const int kbs = (g.K + kLrBK - 1) / kLrBK;
+    const int ntiles = g.m_tiles * g.n_tiles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kLrStages; ++s) {
             lr_mbar_init(&full[s], 1);
             lr_mbar_init(&empty[s], 1);
         }
-        lr_mbar_init(&done, 1);
+        for (int b = 0; b < 2; ++b) {
+            lr_mbar_init(&tfull[b], 1);
+            lr_mbar_init(&tempty[b], kLrEpiWarps);  // one arrival per epilogue warp
+        }
         s_abort = 0;
         s_consumed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(lr_smem(&s_tmem)),
-                     "r"((uint32_t)BN));
+                     "r"(kCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     lr_fence_before();
@@ -195,64 +212,101 @@ __global__ void __launch_bounds__(kLrThreads, 1)
 
     int issued = 0;
     if (warp == 0 && lane == 0) {
-        // ---- producer
-        for (int kb = 0; kb < kbs; ++kb) {
-            const int s = kb % kLrStages;
-            const unsigned round = (unsigned)(kb / kLrStages);
-            if (kb >= kLrStages && !lr_wait(&empty[s], (round - 1u) & 1u, abort, g.err)) break;
-            unsigned char* st = sm + s * STAGE;
-            lr_expect_tx(&full[s], (unsigned)STAGE);
-            lr_tma_2d(st, &ta, &full[s], kb * kLrBK, m_tile * kLrBM);
-            lr_tma_2d(st + A_BYTES, &tb, &full[s], kb * kLrBK, n_tile * BN);
-            issued = kb + 1;
+        // ---- producer: one global count of stages across the CTA's tiles
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const int m_tile = t % g.m_tiles, n_tile = t / g.m_tiles;
+            for (int kb = 0; kb < kbs; ++kb, ++it) {
+                const int s = it % kLrStages;
+                const unsigned ph = (unsigned)(it / kLrStages);
+                if (it >= kLrStages && !lr_wait(&empty[s], (ph - 1u) & 1u, abort, g.err)) { ok = false; break; }
+                unsigned char* st = sm + s * STAGE;
+                lr_expect_tx(&full[s], (unsigned)STAGE);
+                lr_tma_2d(st, &ta, &full[s], kb * kLrBK, m_tile * kLrBM);
+                lr_tma_2d(st + A_BYTES, &tb, &full[s], kb * kLrBK, n_tile * BN);
+                issued = it + 1;
+            }
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer
         constexpr uint32_t idesc = lr_idesc<BN>();
-        for (int kb = 0; kb < kbs; ++kb) {
-            const int s = kb % kLrStages;
-            const unsigned round = (unsigned)(kb / kLrStages);
-            if (!lr_wait(&full[s], round & 1u, abort, g.err)) break;
+        int it = 0, i = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
+            const int b = i & 1, use = i >> 1;
+            if (use >= 1 && !lr_wait(&tempty[b], (unsigned)(use - 1) & 1u, abort, g.err)) break;
             lr_fence_after();
-            const uint32_t a0 = lr_smem(sm + s * STAGE), b0 = a0 + A_BYTES;
+            const uint32_t d = tmem + (uint32_t)(b * BN);
+            for (int kb = 0; kb < kbs; ++kb, ++it) {
+                const int s = it % kLrStages;
+                const unsigned ph = (unsigned)(it / kLrStages);
+                if (!lr_wait(&full[s], ph & 1u, abort, g.err)) { ok = false; break; }
+                lr_fence_after();
+                const uint32_t a0 = lr_smem(sm + s * STAGE), b0 = a0 + A_BYTES;
 #pragma unroll
-            for (int j = 0; j < kLrBK / 16; ++j)  // K = 16 per MMA: 32 bytes along the swizzled row
-                lr_mma(tmem, lr_desc(a0 + 32 * j), lr_desc(b0 + 32 * j), idesc, (kb > 0 || j > 0) ? 1u : 0u);
-            lr_commit(&empty[s]);
-            s_consumed = kb + 1;
+                for (int j = 0; j < kLrBK / 16; ++j)  // K = 16 per MMA: 32 bytes along the swizzled row
+                    lr_mma(d, lr_desc(a0 + 32 * j), lr_desc(b0 + 32 * j), idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                lr_commit(&empty[s]);
+                s_consumed = it + 1;
+            }
+            lr_commit(&tfull[b]);
         }
-        lr_commit(&done);
     } else if (warp >= 4) {
-        // ---- epilogue: warp 4 + q owns TMEM lanes (= tile rows) 32q .. 32q + 31
-        const int q = warp - 4;
-        const int row = m_tile * kLrBM + 32 * q + lane;
-        const bool row_ok = row < g.M;
+        // ---- epilogue: warp 4 + w owns TMEM lanes (= tile rows) 32q .. 32q + 31,
+        // q = w % 4, and the columns of half w / 4
+        const int q = (warp - 4) & 3, half = (warp - 4) >> 2;
+        // a tcgen05.ld reads 32 columns: with BN = 32 the second half of the warps
+        // reads nothing, but still waits and hands back each accumulator (the
+        // barrier counts every epilogue warp)
+        constexpr int HALF = BN >= 64 ? BN / 2 : BN;
+        const bool active = BN >= 64 || half == 0;
         const bool lse = g.part != nullptr;
-        float T = 1.f;
-        if (lse && g.temperature && row_ok) T = g.temperature[row];
-        const bool lse_row = lse && row_ok && T > 0.f && T <= FLT_MAX;
-        float khi = 0.f, klo = 0.f;
-        if (lse_row) split_k(T, &khi, &klo);
-        Lse L;
-        lse_init(L);
-        // one lane waits, so the warp-wide tcgen05.ld below runs on all lanes or none
-        int ready = 0;
-        if (lane == 0) ready = lr_wait(&done, 0u, abort, g.err) ? 1 : 0;
-        ready = __shfl_sync(0xffffffffu, ready, 0);
-        if (ready) {
+        int i = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+            const int m_tile = t % g.m_tiles, n_tile = t / g.m_tiles;
+            const int b = i & 1, use = i >> 1;
+            const int row = m_tile * kLrBM + 32 * q + lane;
+            const bool row_ok = row < g.M;
+            float T = 1.f;
+            if (lse && g.temperature && row_ok) T = g.temperature[row];
+            const bool lse_row = lse && row_ok && T > 0.f && T <= FLT_MAX;
+            float khi = 0.f, klo = 0.f;
+            if (lse_row) split_k(T, &khi, &klo);
+            Lse L;
+            lse_init(L);
+            // one lane waits, so the warp-wide tcgen05.ld below runs on all lanes or none
+            int ready = 0;
+            if (lane == 0) ready = lr_wait(&tfull[b], (unsigned)use & 1u, abort, g.err) ? 1 : 0;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (!ready) break;
             lr_fence_after();
-            for (int c = 0; c < BN; c += 32) {
+            if (!active) {
+                __syncwarp();
+                if (lane == 0) lr_arrive(&tempty[b]);
+                if (lse && row_ok)
+                    g.part[((size_t)row * g.n_tiles + n_tile) * 2 + half] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+                continue;
+            }
+            const uint32_t tb_addr = tmem + (uint32_t)(b * BN + half * HALF) + ((uint32_t)(32 * q) << 16);
+            for (int c = 0; c < HALF; c += 32) {
                 uint32_t r[32];
-                lr_tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, r);
-                const int n0 = n_tile * BN + c;
+                lr_tmem_ld32(tb_addr + (uint32_t)c, r);
+                if (c + 32 == HALF) {
+                    // this warp's part of the accumulator is read: hand it back
+                    lr_fence_before();
+                    __syncwarp();
+                    if (lane == 0) lr_arrive(&tempty[b]);
+                }
+                const int n0 = n_tile * BN + half * HALF + c;
                 float x[32];
                 uint32_t packed[16];
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-                    packed[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-                    x[i] = __bfloat162float(h2.x);
-                    x[i + 1] = __bfloat162float(h2.y);
+                for (int k = 0; k < 32; k += 2) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[k]), __uint_as_float(r[k + 1]));
+                    packed[k / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                    x[k] = __bfloat162float(h2.x);
+                    x[k + 1] = __bfloat162float(h2.y);
                 }
                 if (row_ok) {
                     __nv_bfloat16* dst = g.out + (size_t)row * g.N + n0;
@@ -262,37 +316,48 @@ __global__ void __launch_bounds__(kLrThreads, 1)
                             reinterpret_cast<uint4*>(dst)[v] =
                                 make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                     } else {
-                        for (int i = 0; i < 32 && n0 + i < g.N; ++i) {
-                            const uint32_t w = packed[i / 2];
-                            const unsigned short hb = (unsigned short)((i & 1) ? (w >> 16) : (w & 0xffffu));
-                            reinterpret_cast<unsigned short*>(dst)[i] = hb;
+                        for (int k = 0; k < 32 && n0 + k < g.N; ++k) {
+                            const uint32_t w = packed[k / 2];
+                            reinterpret_cast<unsigned short*>(dst)[k] =
+                                (unsigned short)((k & 1) ? (w >> 16) : (w & 0xffffu));
                         }
                     }
                 }
                 if (lse_row) {
+                    // one maximum and at most one rescale per 32 columns, then 32
+                    // independent terms into 8 accumulators
+                    float vm = -INFINITY;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (n0 + i >= g.N) x[i] = -INFINITY;  // columns past N take no part
+                    for (int k = 0; k < 32; ++k) {
+                        if (n0 + k >= g.N) x[k] = -INFINITY;  // columns past N take no part
+                        vm = fmaxf(vm, x[k]);
+                    }
+                    lse_rebase(L, vm, khi);
+                    float acc[8];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) lse_add<8>(L, x + i, khi, klo);
+                    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) acc[k & 7] += scaled_exp(x[k], khi, klo, L.mk);
+                    L.s += tree8(acc);
                 }
             }
+            if (lse && row_ok)
+                g.part[((size_t)row * g.n_tiles + n_tile) * 2 + half] = make_float4(L.m, L.mk, L.s, 0.f);
         }
-        if (lse && row_ok) g.part[(size_t)row * g.n_tiles + n_tile] = make_float4(L.m, L.mk, L.s, 0.f);
     }
     lr_fence_before();
     __syncthreads();
     // after a wait gave up: let the copies this CTA issued but never consumed land
     // (bounded) before its shared memory goes away
     if (warp == 0 && lane == 0 && s_abort)
-        for (int kb = s_consumed; kb < issued; ++kb) {
-            const unsigned par = (unsigned)(kb / kLrStages) & 1u;
-            for (unsigned i = 0; i < kLrSpin && !lr_try_wait(&full[kb % kLrStages], par); ++i) {
+        for (int it = s_consumed; it < issued; ++it) {
+            const unsigned par = (unsigned)(it / kLrStages) & 1u;
+            for (unsigned k = 0; k < kLrSpin && !lr_try_wait(&full[it % kLrStages], par); ++k) {
             }
         }
     if (warp == 2) {
         lr_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)BN));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
     }
 }
 
