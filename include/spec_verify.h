@@ -437,7 +437,8 @@ sv_status spec_verify_lowrank_down(const void* h, const void* w_down, int M, int
                                    int32_t* out_error, struct CUstream_st* stream);
 
 /* z = bf16(u W_up^T): [M][V], and (if out_lse) each row's log-normaliser; the
- * workspace (256-byte aligned) holds 2 M ceil(V / 256) partials of 16 bytes. */
+ * workspace (256-byte aligned) holds the normaliser partials:
+ * spec_verify_lowrank_workspace_size(M, r, V) minus the u part. */
 sv_status spec_verify_lowrank_up(const void* u, const void* w_up, int M, int r, int V, const float* temperature,
                                  void* out_logits, double* out_lse, void* workspace, size_t workspace_bytes,
                                  int32_t* out_error, struct CUstream_st* stream);

@@ -24,6 +24,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <cstring>
 
 #include "sv_common.cuh"
 #include "sv_generic.cuh"
@@ -810,18 +811,19 @@ TensorMapEncodeFn tensor_map_encoder()
     return fn;
 }
 
-// Tensor map of a row-major [rows][K] bf16 matrix, loaded as boxes of 64 (K) x
-// box_rows with the 128-byte swizzle; out-of-range elements read as zero.
-bool lr_map(CUtensorMap* m, const void* base, long long rows, long long K, int box_rows)
+// Tensor map of a row-major [rows][K] bf16 matrix, in boxes of box_k (K) x
+// box_rows; out-of-range elements read as zero and are not written.
+bool lr_map(CUtensorMap* m, const void* base, long long rows, long long K, int box_rows, int box_k = sv::kLrBK,
+            CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     TensorMapEncodeFn enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)sv::kLrBK, (cuuint32_t)box_rows};
+    const cuuint32_t box[2] = {(cuuint32_t)box_k, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -829,16 +831,19 @@ template <int BN>
 cudaError_t lr_launch(const void* A, const void* B, int M, int N, int K, void* out, float4* part,
                       const float* temperature, int* err, cudaStream_t st)
 {
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
     if (!lr_map(&ta, A, M, K, sv::kLrBM) || !lr_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
-    constexpr int smem = sv::lr_smem_bytes<BN>();
+    // the output goes out through TMA stores when its rows are 16-byte multiples
+    const bool tma_store = (N % 8) == 0 && lr_map(&tc, out, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!tma_store) memset(&tc, 0, sizeof tc);
     static std::once_flag once[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     cudaError_t attr_err = cudaSuccess;
     if (dev >= 0 && dev < kMaxDevices)
         std::call_once(once[dev], [&] {
-            attr_err = cudaFuncSetAttribute(sv::sv_lr_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            attr_err = cudaFuncSetAttribute(sv::sv_lr_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            sv::kLrSmemMax);
         });
     if (attr_err != cudaSuccess) return attr_err;
     sv::LrArgs g;
@@ -851,8 +856,27 @@ cudaError_t lr_launch(const void* A, const void* B, int M, int N, int K, void* o
     g.n_tiles = (int)cdiv(N, BN);
     const long long tiles = (long long)g.m_tiles * g.n_tiles;
     if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const long long grid = std::min<long long>(tiles, device_sm_count());  // one CTA per SM (shared memory)
-    sv::sv_lr_gemm<BN><<<(unsigned)grid, sv::kLrThreads, smem, st>>>(ta, tb, g);
+    const int sms = device_sm_count();
+    const long long kbs = cdiv(K, sv::kLrBK);
+    const long long a_bytes = (long long)sv::kLrBM * sv::kLrBK * 2, b_bytes = (long long)BN * sv::kLrBK * 2;
+    const long long budget = sv::kLrSmemMax - 1024 - (tma_store ? sv::kLrStagingBytes : 0);
+    // A resident: its K blocks plus at least 3 stages of B fit, and every row tile
+    // gets at least one CTA
+    g.tma_store = tma_store ? 1 : 0;
+    g.a_resident = (kbs <= sv::kLrMaxResidentKb && kbs * a_bytes + 3 * b_bytes <= budget && g.m_tiles <= sms) ? 1 : 0;
+    const long long stage = g.a_resident ? b_bytes : a_bytes + b_bytes;
+    const long long room = budget - (g.a_resident ? kbs * a_bytes : 0);
+    g.stages = (int)std::min<long long>(sv::kLrMaxStages, room / stage);
+    long long grid;
+    if (g.a_resident) {
+        const long long slots = std::min<long long>(sms / g.m_tiles, g.n_tiles);
+        grid = slots * g.m_tiles;
+    } else {
+        grid = std::min<long long>(tiles, sms);  // one CTA per SM (shared memory)
+    }
+    const long long smem =
+        1024 + (g.a_resident ? kbs * a_bytes : 0) + g.stages * stage + (tma_store ? sv::kLrStagingBytes : 0);
+    sv::sv_lr_gemm<BN><<<(unsigned)grid, sv::kLrThreads, (size_t)smem, st>>>(ta, tb, tc, g);
     return cudaGetLastError();
 }
 
@@ -867,7 +891,7 @@ constexpr int kLrUpBN = 256;
 constexpr int kLrDownBN = 32;
 
 size_t lr_u_bytes(int M, int r) { return ((size_t)M * r * 2 + 1023) / 1024 * 1024; }
-size_t lr_part_bytes(int M, int V) { return (size_t)M * (size_t)cdiv(V, kLrUpBN) * 2 * sizeof(float4); }
+size_t lr_part_bytes(int M, int V) { return (size_t)M * (size_t)cdiv(V, kLrUpBN) * sv::kLrGroups * sizeof(float4); }
 
 }  // namespace
 
@@ -907,7 +931,7 @@ extern "C" sv_status spec_verify_lowrank_up(const void* u, const void* w_up, int
     if (e != cudaSuccess) return e == cudaErrorInvalidValue ? SV_ERR_INVALID_ARG : SV_ERR_CUDA;
     if (out_lse) {
         sv::sv_lr_lse<<<(unsigned)cdiv((long long)M * 32, 256), 256, 0, st>>>(part, temperature, M,
-                                                                            2 * (int)cdiv(V, kLrUpBN), out_lse);
+                                                                            sv::kLrGroups * (int)cdiv(V, kLrUpBN), out_lse);
         if (cudaGetLastError() != cudaSuccess) return SV_ERR_CUDA;
     }
     return SV_OK;

@@ -12,9 +12,11 @@
 // arithmetic of the verifier's passes), written as one partial per (row,
 // column tile) and folded by sv_lr_lse.
 //
-// sv_lr_gemm: persistent, one CTA per SM walking 128 x BN output tiles (column
-// tiles outer, so the row tiles sharing a W tile run together and read it once
-// from HBM), the accumulator double-buffered in TMEM.
+// sv_lr_gemm: persistent, one CTA per SM walking 128 x BN output tiles, the
+// accumulator double-buffered in TMEM.  When K fits (K <= 512, the up contraction
+// with r <= 512), a CTA keeps one row tile of A (all of K) in shared memory and
+// streams only B; the CTAs of a slot walk the same column tiles, so each W tile
+// comes from HBM once.  Otherwise both operands stream through the ring.
 //   warp 0 (one thread)  TMA: 128 x 64 of A and BN x 64 of B per stage, 128-byte
 //                        swizzle, kLrStages stages, mbarrier transaction counts
 //   warp 1 (one thread)  tcgen05.mma kind::f16 (bf16 x bf16 -> f32), M = 128,
@@ -23,10 +25,10 @@
 //                        stage signals the epilogue
 //   warp 2               allocates and frees the TMEM columns
 //   warps 4-11           epilogue: tcgen05.ld of 32 lanes x 32 columns at a
-//                        time (warp 4 + w reads lanes 32 (w % 4) ... + 31 and
-//                        columns half w / 4), bf16 rounding, 16-byte stores, the
-//                        row's online log-sum-exp over its half of the columns
-// Every wait on an mbarrier is bounded: past kLrSpin polls the CTA raises
+//                        time (warp 4 + w reads lanes 32 (w % 4) ... + 31 and the
+//                        columns of group w / 4), bf16 rounding, 16-byte stores,
+//                        the row's online log-sum-exp over its group
+// Every wait on an mbarrier is bounded: past kLrPolls polls the CTA raises
 // *err, stops issuing, and still frees its TMEM.
 #pragma once
 
@@ -39,19 +41,27 @@ namespace sv {
 
 constexpr int kLrBM = 128;      // tile rows = the MMA's M
 constexpr int kLrBK = 64;       // K per stage: one 128-byte swizzled row of bf16
-constexpr int kLrStages = 4;
-constexpr int kLrEpiWarps = 8;  // two per TMEM lane quarter, each on half the columns
+constexpr int kLrMaxStages = 4;
+constexpr int kLrMaxResidentKb = 8;  // A stays in shared memory when K <= 8 x 64
+constexpr int kLrEpiWarps = 8;   // per TMEM lane quarter kLrGroups warps, each on a column group
+constexpr int kLrGroups = kLrEpiWarps / 4;
 constexpr int kLrThreads = 128 + 32 * kLrEpiWarps;
-constexpr unsigned kLrSpin = 1u << 24;
+constexpr int kLrSmemMax = 227 * 1024 - 1024;  // dynamic shared memory of one CTA (static part kept apart)
 
 struct LrArgs {
     __nv_bfloat16* out;        // [M][N]
-    float4* part;              // [M][2 n_tiles] (m, mk, s, 0) per column half, or null
+    float4* part;              // [M][kLrGroups n_tiles] (m, mk, s, 0) per column group, or null
     const float* temperature;  // [M] or null (T = 1)
     int* err;                  // optional: 1 if a wait gave up
     int M, N, K;
     int m_tiles, n_tiles;
+    int stages;                // ring depth
+    int a_resident;            // the CTA's A tile (all of K) is loaded once and kept
+    int tma_store;             // out written by TMA stores of 32 x 32 chunks staged in shared memory
 };
+
+constexpr int kLrChunkBytes = 32 * 32 * 2;                      // one 32-row x 32-column bf16 chunk
+constexpr int kLrStagingBytes = kLrEpiWarps * 2 * kLrChunkBytes;  // two chunks per epilogue warp
 
 __device__ __forceinline__ uint32_t lr_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -65,30 +75,46 @@ __device__ __forceinline__ void lr_expect_tx(uint64_t* bar, unsigned bytes)
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(lr_smem(bar)), "r"(bytes) : "memory");
 }
 
+// One poll that may suspend the thread for up to kLrPollNs while the phase is
+// still open (it returns as soon as the phase completes), so waiting warps take
+// no issue slots from the producer and the MMA thread.
+constexpr unsigned kLrPollNs = 20000;
+constexpr unsigned kLrPolls = 200000;  // with the suspension: seconds, not hours
+
 __device__ __forceinline__ bool lr_try_wait(uint64_t* bar, unsigned parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(lr_smem(bar)), "r"(parity)
+        : "r"(lr_smem(bar)), "r"(parity), "r"(kLrPollNs)
         : "memory");
     return ok != 0;
 }
 
 // Wait for the phase with this parity; false (after raising the flags) if it did
-// not complete within kLrSpin polls, or another role of the CTA already gave up.
+// not complete within kLrPolls polls, or another role of the CTA already gave up.
 __device__ __forceinline__ bool lr_wait(uint64_t* bar, unsigned parity, volatile int* abort, int* err)
 {
-    for (unsigned i = 0; i < kLrSpin; ++i) {
+    for (unsigned i = 0; i < kLrPolls; ++i) {
         if (lr_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 1023u && *abort) return false;
+        if ((i & 63u) == 63u && *abort) return false;
     }
     *abort = 1;
     if (err) atomicExch(err, 1);
     return false;
+}
+
+// shared -> global tensor store of one staged chunk; rows and columns past the
+// tensor's extent are not written
+__device__ __forceinline__ void lr_tma_store_2d(const CUtensorMap* map, const void* src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"((uint64_t)map),
+                 "r"(lr_smem(src)), "r"(x), "r"(y)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
 __device__ __forceinline__ void lr_tma_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y)
@@ -150,44 +176,61 @@ __device__ __forceinline__ void lr_tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-template <int BN>
-constexpr int lr_smem_bytes()
-{
-    return kLrStages * (kLrBM * kLrBK * 2 + BN * kLrBK * 2) + 1024;  // + alignment slack
-}
-
 __device__ __forceinline__ void lr_arrive(uint64_t* bar)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(lr_smem(bar)) : "memory");
 }
 
-// Persistent: CTA c takes tiles c, c + gridDim.x, ... (consecutive tiles share a
-// column tile, so the row tiles of one W tile run at the same time).  The
-// accumulator is double-buffered in TMEM (2 x BN columns): while the epilogue
-// warps drain tile i from one buffer, the MMA thread fills the other with tile
-// i + 1, and the producer keeps loading ahead through the stage ring.
+// The k-th tile of CTA c, or false past its last.  A resident: the CTA keeps
+// row tile c % m_tiles and walks column tiles slot, slot + nslots, ... (the
+// CTAs of one slot run the same column tile at about the same time, so its W
+// rows come from HBM once); otherwise tiles c, c + gridDim.x, ... with the row
+// tile fastest.
+__device__ __forceinline__ bool lr_tile(const LrArgs& g, int k, int* m, int* n)
+{
+    if (g.a_resident) {
+        const int nslots = (int)gridDim.x / g.m_tiles;
+        *m = (int)blockIdx.x % g.m_tiles;
+        *n = (int)blockIdx.x / g.m_tiles + k * nslots;
+        return *n < g.n_tiles;
+    }
+    const long long t = (long long)blockIdx.x + (long long)k * gridDim.x;
+    if (t >= (long long)g.m_tiles * g.n_tiles) return false;
+    *m = (int)(t % g.m_tiles);
+    *n = (int)(t / g.m_tiles);
+    return true;
+}
+
+// Persistent, one CTA per SM; the accumulator is double-buffered in TMEM (2 x BN
+// columns): while the epilogue warps drain tile i from one buffer, the MMA thread
+// fills the other with tile i + 1, and the producer keeps loading ahead through
+// the stage ring.
 template <int BN>
 __global__ void __launch_bounds__(kLrThreads, 1)
-    sv_lr_gemm(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, LrArgs g)
+    sv_lr_gemm(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+               const __grid_constant__ CUtensorMap tc, LrArgs g)
 {
     static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "tile columns: a power of two TMEM allocation");
-    constexpr int A_BYTES = kLrBM * kLrBK * 2;
+    constexpr int A_BYTES = kLrBM * kLrBK * 2;  // one K block of A
     constexpr int B_BYTES = BN * kLrBK * 2;
-    constexpr int STAGE = A_BYTES + B_BYTES;
-    constexpr uint32_t kCols = 2 * BN;  // two accumulators
+    constexpr uint32_t kCols = 2 * BN;          // two accumulators
     extern __shared__ unsigned char lr_dyn[];
-    // the stages start on a 1024-byte boundary of the shared window (the swizzle atom)
+    // every tile starts on a 1024-byte boundary of the shared window (the swizzle atom)
     unsigned char* sm = lr_dyn + ((1024u - (lr_smem(lr_dyn) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t full[kLrStages], empty[kLrStages], tfull[2], tempty[2];
+    __shared__ __align__(8) uint64_t full[kLrMaxStages], empty[kLrMaxStages], tfull[2], tempty[2], afull;
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort, s_consumed;
+    __shared__ int s_abort, s_consumed, s_a_done;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kbs = (g.K + kLrBK - 1) / kLrBK;
-    const int ntiles = g.m_tiles * g.n_tiles;
+    const bool res = g.a_resident != 0;
+    const int S = g.stages;
+    const int STAGE = res ? B_BYTES : A_BYTES + B_BYTES;
+    unsigned char* ring = sm + (res ? kbs * A_BYTES : 0);
+    unsigned char* staging = ring + S * STAGE;  // tma_store: kLrStagingBytes after the ring
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kLrStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             lr_mbar_init(&full[s], 1);
             lr_mbar_init(&empty[s], 1);
         }
@@ -195,8 +238,10 @@ __global__ void __launch_bounds__(kLrThreads, 1)
             lr_mbar_init(&tfull[b], 1);
             lr_mbar_init(&tempty[b], kLrEpiWarps);  // one arrival per epilogue warp
         }
+        lr_mbar_init(&afull, 1);
         s_abort = 0;
         s_consumed = 0;
+        s_a_done = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 2) {
@@ -210,40 +255,51 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     const uint32_t tmem = s_tmem;
     volatile int* abort = &s_abort;
 
-    int issued = 0;
+    int issued = 0, a_issued = 0;
     if (warp == 0 && lane == 0) {
         // ---- producer: one global count of stages across the CTA's tiles
-        int it = 0;
+        int m0, n0;
+        if (res && lr_tile(g, 0, &m0, &n0)) {
+            lr_expect_tx(&afull, (unsigned)(kbs * A_BYTES));
+            for (int kb = 0; kb < kbs; ++kb) lr_tma_2d(sm + kb * A_BYTES, &ta, &afull, kb * kLrBK, m0 * kLrBM);
+            a_issued = 1;
+        }
+        int it = 0, m, n;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const int m_tile = t % g.m_tiles, n_tile = t / g.m_tiles;
+        for (int k = 0; ok && lr_tile(g, k, &m, &n); ++k) {
             for (int kb = 0; kb < kbs; ++kb, ++it) {
-                const int s = it % kLrStages;
-                const unsigned ph = (unsigned)(it / kLrStages);
-                if (it >= kLrStages && !lr_wait(&empty[s], (ph - 1u) & 1u, abort, g.err)) { ok = false; break; }
-                unsigned char* st = sm + s * STAGE;
+                const int s = it % S;
+                const unsigned ph = (unsigned)(it / S);
+                if (it >= S && !lr_wait(&empty[s], (ph - 1u) & 1u, abort, g.err)) { ok = false; break; }
+                unsigned char* st = ring + s * STAGE;
                 lr_expect_tx(&full[s], (unsigned)STAGE);
-                lr_tma_2d(st, &ta, &full[s], kb * kLrBK, m_tile * kLrBM);
-                lr_tma_2d(st + A_BYTES, &tb, &full[s], kb * kLrBK, n_tile * BN);
+                if (!res) lr_tma_2d(st, &ta, &full[s], kb * kLrBK, m * kLrBM);
+                lr_tma_2d(st + (res ? 0 : A_BYTES), &tb, &full[s], kb * kLrBK, n * BN);
                 issued = it + 1;
             }
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer
         constexpr uint32_t idesc = lr_idesc<BN>();
-        int it = 0, i = 0;
+        int it = 0, i = 0, m, n;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
+        if (res && lr_tile(g, 0, &m, &n)) {
+            ok = lr_wait(&afull, 0u, abort, g.err);
+            s_a_done = ok ? 1 : 0;
+        }
+        for (; ok && lr_tile(g, i, &m, &n); ++i) {
             const int b = i & 1, use = i >> 1;
             if (use >= 1 && !lr_wait(&tempty[b], (unsigned)(use - 1) & 1u, abort, g.err)) break;
             lr_fence_after();
             const uint32_t d = tmem + (uint32_t)(b * BN);
             for (int kb = 0; kb < kbs; ++kb, ++it) {
-                const int s = it % kLrStages;
-                const unsigned ph = (unsigned)(it / kLrStages);
+                const int s = it % S;
+                const unsigned ph = (unsigned)(it / S);
                 if (!lr_wait(&full[s], ph & 1u, abort, g.err)) { ok = false; break; }
                 lr_fence_after();
-                const uint32_t a0 = lr_smem(sm + s * STAGE), b0 = a0 + A_BYTES;
+                const uint32_t st = lr_smem(ring + s * STAGE);
+                const uint32_t a0 = res ? lr_smem(sm + kb * A_BYTES) : st;
+                const uint32_t b0 = res ? st : st + A_BYTES;
 #pragma unroll
                 for (int j = 0; j < kLrBK / 16; ++j)  // K = 16 per MMA: 32 bytes along the swizzled row
                     lr_mma(d, lr_desc(a0 + 32 * j), lr_desc(b0 + 32 * j), idesc, (kb > 0 || j > 0) ? 1u : 0u);
@@ -254,27 +310,21 @@ __global__ void __launch_bounds__(kLrThreads, 1)
         }
     } else if (warp >= 4) {
         // ---- epilogue: warp 4 + w owns TMEM lanes (= tile rows) 32q .. 32q + 31,
-        // q = w % 4, and the columns of half w / 4
-        const int q = (warp - 4) & 3, half = (warp - 4) >> 2;
-        // a tcgen05.ld reads 32 columns: with BN = 32 the second half of the warps
-        // reads nothing, but still waits and hands back each accumulator (the
-        // barrier counts every epilogue warp)
-        constexpr int HALF = BN >= 64 ? BN / 2 : BN;
-        const bool active = BN >= 64 || half == 0;
+        // q = w % 4, and column group w / 4 (QCOLS columns; a tcgen05.ld reads 32, so
+        // with BN < 128 the groups past BN read nothing but still wait for and hand
+        // back each accumulator: the barrier counts every epilogue warp)
+        const int q = (warp - 4) & 3, grp = (warp - 4) >> 2;
+        constexpr int QCOLS = BN / kLrGroups >= 32 ? BN / kLrGroups : 32;
+        const bool active = grp * QCOLS < BN;
         const bool lse = g.part != nullptr;
-        int i = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
-            const int m_tile = t % g.m_tiles, n_tile = t / g.m_tiles;
+        unsigned char* stg = staging + (warp - 4) * 2 * kLrChunkBytes;
+        int chunks = 0;  // chunks this warp has staged (the buffer alternates)
+        int i = 0, m_tile, n_tile;
+        for (; lr_tile(g, i, &m_tile, &n_tile); ++i) {
             const int b = i & 1, use = i >> 1;
             const int row = m_tile * kLrBM + 32 * q + lane;
             const bool row_ok = row < g.M;
-            float T = 1.f;
-            if (lse && g.temperature && row_ok) T = g.temperature[row];
-            const bool lse_row = lse && row_ok && T > 0.f && T <= FLT_MAX;
-            float khi = 0.f, klo = 0.f;
-            if (lse_row) split_k(T, &khi, &klo);
-            Lse L;
-            lse_init(L);
+            float4* part = (lse && row_ok) ? g.part + ((size_t)row * g.n_tiles + n_tile) * kLrGroups + grp : nullptr;
             // one lane waits, so the warp-wide tcgen05.ld below runs on all lanes or none
             int ready = 0;
             if (lane == 0) ready = lr_wait(&tfull[b], (unsigned)use & 1u, abort, g.err) ? 1 : 0;
@@ -284,21 +334,27 @@ __global__ void __launch_bounds__(kLrThreads, 1)
             if (!active) {
                 __syncwarp();
                 if (lane == 0) lr_arrive(&tempty[b]);
-                if (lse && row_ok)
-                    g.part[((size_t)row * g.n_tiles + n_tile) * 2 + half] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+                if (part) *part = make_float4(-INFINITY, 0.f, 0.f, 0.f);
                 continue;
             }
-            const uint32_t tb_addr = tmem + (uint32_t)(b * BN + half * HALF) + ((uint32_t)(32 * q) << 16);
-            for (int c = 0; c < HALF; c += 32) {
+            float T = 1.f;
+            if (part && g.temperature) T = g.temperature[row];
+            const bool lse_row = part != nullptr && T > 0.f && T <= FLT_MAX;
+            float khi = 0.f, klo = 0.f;
+            if (lse_row) split_k(T, &khi, &klo);
+            Lse L;
+            lse_init(L);
+            const uint32_t tb_addr = tmem + (uint32_t)(b * BN + grp * QCOLS) + ((uint32_t)(32 * q) << 16);
+            for (int c = 0; c < QCOLS; c += 32) {
                 uint32_t r[32];
                 lr_tmem_ld32(tb_addr + (uint32_t)c, r);
-                if (c + 32 == HALF) {
+                if (c + 32 == QCOLS) {
                     // this warp's part of the accumulator is read: hand it back
                     lr_fence_before();
                     __syncwarp();
                     if (lane == 0) lr_arrive(&tempty[b]);
                 }
-                const int n0 = n_tile * BN + half * HALF + c;
+                const int n0 = n_tile * BN + grp * QCOLS + c;
                 float x[32];
                 uint32_t packed[16];
 #pragma unroll
@@ -308,7 +364,23 @@ __global__ void __launch_bounds__(kLrThreads, 1)
                     x[k] = __bfloat162float(h2.x);
                     x[k + 1] = __bfloat162float(h2.y);
                 }
-                if (row_ok) {
+                if (g.tma_store) {
+                    // stage the warp's 32 x 32 chunk (lane = row, 64 bytes each) and
+                    // let one TMA store write it
+                    unsigned char* buf = stg + (chunks & 1) * kLrChunkBytes;
+                    if (chunks >= 2) {
+                        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        reinterpret_cast<uint4*>(buf + lane * 64)[v] =
+                            make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) lr_tma_store_2d(&tc, buf, n0, m_tile * kLrBM + 32 * q);
+                    ++chunks;
+                } else if (row_ok) {
                     __nv_bfloat16* dst = g.out + (size_t)row * g.N + n0;
                     if (n0 + 32 <= g.N && (g.N & 7) == 0) {
 #pragma unroll
@@ -341,20 +413,26 @@ __global__ void __launch_bounds__(kLrThreads, 1)
                     L.s += tree8(acc);
                 }
             }
-            if (lse && row_ok)
-                g.part[((size_t)row * g.n_tiles + n_tile) * 2 + half] = make_float4(L.m, L.mk, L.s, 0.f);
+            if (part) *part = make_float4(L.m, L.mk, L.s, 0.f);
         }
+        // the staged chunks are written before the CTA (and its shared memory) ends
+        if (g.tma_store && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
     }
     lr_fence_before();
     __syncthreads();
     // after a wait gave up: let the copies this CTA issued but never consumed land
     // (bounded) before its shared memory goes away
-    if (warp == 0 && lane == 0 && s_abort)
+    if (warp == 0 && lane == 0 && s_abort) {
+        if (a_issued && !s_a_done)
+            for (unsigned k = 0; k < kLrPolls && !lr_try_wait(&afull, 0u); ++k) {
+            }
         for (int it = s_consumed; it < issued; ++it) {
-            const unsigned par = (unsigned)(it / kLrStages) & 1u;
-            for (unsigned k = 0; k < kLrSpin && !lr_try_wait(&full[it % kLrStages], par); ++k) {
+            const unsigned par = (unsigned)(it / S) & 1u;
+            for (unsigned k = 0; k < kLrPolls && !lr_try_wait(&full[it % S], par); ++k) {
             }
         }
+    }
     if (warp == 2) {
         lr_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
