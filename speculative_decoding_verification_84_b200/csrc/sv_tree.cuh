@@ -386,13 +386,18 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         // ---- the children, in index order
         const double Td = (double)T;
         int level = 0, next = -1, k = 0;
+        // set when the last child's rejection applied its residual: the draw's
+        // weights are that residual, so its sums (sm.wsum, sm.x[reuse_par]) stand
+        int reuse_par = -1;
         for (int i = sm.first_child[c]; i >= 0; i = sm.next_sib[i], ++k) {
             const double lq = (double)sm.ld[k] / Td - a2d * kLn2;
             const double lp = level == 0 ? (double)sm.lt[k] / Td - a2t * kLn2
                                          : log((double)tree_weight(rw, sm.inv_S, level, false, sm.lt[k], sm.ld[k]));
             if (log((double)a.u_accept[(size_t)b * N + i]) < lp - lq) { next = i; break; }
-            // rejected: the mass of max(0, P - q)
+            // rejected: the mass of max(0, P - q) (and its last positive token, for
+            // a draw that may reuse these sums)
             double part = 0.0;
+            int last = -1;
             for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
                 uint4 rt[kTreeBatch], rd[kTreeBatch];
 #pragma unroll
@@ -408,31 +413,40 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
                         unpack<ESZ>(rt[u], xt);
                         unpack<ESZ>(rd[u], xd);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
+                        for (int e = 0; e < 8; ++e) {
                             wv[e] = e < VEC ? tree_weight(rw, sm.inv_S, level, true, xt[e], xd[e]) : 0.f;
+                            if (e < VEC && wv[e] > 0.f) last = (int)((g0 + 32 * u) * VEC + e);
+                        }
                         part += (double)tree8(wv);
                     }
             }
             part = warp_sum(part);
-            if (lane == 0) sm.wsum[warp] = part;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+            if (lane == 0) { sm.wsum[warp] = part; sm.wlast[warp] = last; }
             __syncthreads();
             if (tid == 0) {
                 double s = 0.0;
-                for (int w = 0; w < kTreeWarps; ++w) s += sm.wsum[w];
+                int l = -1;
+                for (int w = 0; w < kTreeWarps; ++w) { s += sm.wsum[w]; l = max(l, sm.wlast[w]); }
                 TreeSlot t{};
                 t.s[0] = s;
+                t.idx = l;
                 s_mine = t;
             }
             __syncthreads();
             tree_exchange(cl, sm, xpar, s_mine, CL, rank);
             double S = 0.0;
             for (int q = 0; q < CL; ++q) S += sm.x[xpar][q].s[0];
+            const int this_par = xpar;
             xpar ^= 1;
             if (S < kResidualMin || S != S) {
                 st |= SV_ROW_RESIDUAL_ZERO;  // the residual vanished: P stays
+                reuse_par = -1;
             } else {
                 if (tid == 0) sm.inv_S[level] = (float)(1.0 / S);
                 ++level;
+                reuse_par = sm.next_sib[i] < 0 ? this_par : -1;
             }
             __syncthreads();
         }
@@ -447,49 +461,54 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         // ---- the extra token from P: p (no rejection) or the last residual
         const bool resid = level > 0;
         const int lev = resid ? level - 1 : 0;
-        double part = 0.0;
-        int last = -1;
-        for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
-            uint4 rt[kTreeBatch], rd[kTreeBatch];
+        int dpar = reuse_par;
+        if (dpar < 0) {
+            double part = 0.0;
+            int last = -1;
+            for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
+                uint4 rt[kTreeBatch], rd[kTreeBatch];
 #pragma unroll
-            for (int u = 0; u < kTreeBatch; ++u)
-                if (g0 + 32 * u < hi) {
-                    rt[u] = tree_raw<ESZ, VEC16>(trow, g0 + 32 * u, V);
-                    rd[u] = resid ? tree_raw<ESZ, VEC16>(drow, g0 + 32 * u, V) : rt[u];
-                }
-#pragma unroll
-            for (int u = 0; u < kTreeBatch; ++u)
-                if (g0 + 32 * u < hi) {
-                    float xt[VEC], xd[VEC], wv[8];
-                    unpack<ESZ>(rt[u], xt);
-                    unpack<ESZ>(rd[u], xd);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        wv[e] = e < VEC ? tree_weight(rw, sm.inv_S, lev, resid, xt[e], xd[e]) : 0.f;
-                        if (e < VEC && wv[e] > 0.f) last = (int)((g0 + 32 * u) * VEC + e);
+                for (int u = 0; u < kTreeBatch; ++u)
+                    if (g0 + 32 * u < hi) {
+                        rt[u] = tree_raw<ESZ, VEC16>(trow, g0 + 32 * u, V);
+                        rd[u] = resid ? tree_raw<ESZ, VEC16>(drow, g0 + 32 * u, V) : rt[u];
                     }
-                    part += (double)tree8(wv);
-                }
-        }
-        part = warp_sum(part);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-        if (lane == 0) { sm.wsum[warp] = part; sm.wlast[warp] = last; }
-        __syncthreads();
-        if (tid == 0) {
-            double s = 0.0;
-            int l = -1;
-            for (int w = 0; w < kTreeWarps; ++w) { s += sm.wsum[w]; l = max(l, sm.wlast[w]); }
-            TreeSlot t{};
-            t.s[0] = s;
-            t.idx = l;
-            s_mine = t;
+                for (int u = 0; u < kTreeBatch; ++u)
+                    if (g0 + 32 * u < hi) {
+                        float xt[VEC], xd[VEC], wv[8];
+                        unpack<ESZ>(rt[u], xt);
+                        unpack<ESZ>(rd[u], xd);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            wv[e] = e < VEC ? tree_weight(rw, sm.inv_S, lev, resid, xt[e], xd[e]) : 0.f;
+                            if (e < VEC && wv[e] > 0.f) last = (int)((g0 + 32 * u) * VEC + e);
+                        }
+                        part += (double)tree8(wv);
+                    }
+            }
+            part = warp_sum(part);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+            if (lane == 0) { sm.wsum[warp] = part; sm.wlast[warp] = last; }
+            __syncthreads();
+            if (tid == 0) {
+                double s = 0.0;
+                int l = -1;
+                for (int w = 0; w < kTreeWarps; ++w) { s += sm.wsum[w]; l = max(l, sm.wlast[w]); }
+                TreeSlot t{};
+                t.s[0] = s;
+                t.idx = l;
+                s_mine = t;
+            }
+            __syncthreads();
+            tree_exchange(cl, sm, xpar, s_mine, CL, rank);
+            dpar = xpar;
+            xpar ^= 1;
         }
-        __syncthreads();
-        tree_exchange(cl, sm, xpar, s_mine, CL, rank);
         double S = 0.0;
         int lastpos = -1;
-        for (int q = 0; q < CL; ++q) { S += sm.x[xpar][q].s[0]; lastpos = max(lastpos, sm.x[xpar][q].idx); }
+        for (int q = 0; q < CL; ++q) { S += sm.x[dpar][q].s[0]; lastpos = max(lastpos, sm.x[dpar][q].idx); }
         const double target = (double)a.u_resample[b] * S;
         // the CTA whose range holds the crossing
         int rstar = -1;
@@ -497,12 +516,11 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         {
             double C = 0.0;
             for (int q = 0; q < CL; ++q) {
-                const double s = sm.x[xpar][q].s[0];
+                const double s = sm.x[dpar][q].s[0];
                 if (C + s > target) { rstar = q; before = C; break; }
                 C += s;
             }
         }
-        xpar ^= 1;
         extra = lastpos;  // if rounding leaves no crossing: the last token with a positive weight
         writer = rstar >= 0 ? rstar : 0;
         if (rstar == rank) {
