@@ -196,7 +196,7 @@ def cache_lookup(out_tokens: np.ndarray, out_n: np.ndarray, cache: np.ndarray, F
     return slot
 
 
-BANDIT_UCB1, BANDIT_THOMPSON = 0, 1
+BANDIT_UCB1, BANDIT_THOMPSON, BANDIT_THOMPSON_BETA = 0, 1, 2
 
 
 class Bandit:

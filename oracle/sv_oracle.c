@@ -495,9 +495,13 @@ int sv_oracle_cache_lookup(const int32_t* out_tokens, const int32_t* out_n, cons
  *   Thompson sampling with Gaussian posteriors (Agrawal and Goyal, 2013):
  *     argmax_k R_k/N_k + z_k / sqrt(N_k + 1), z_k = sqrt(-2 ln(1 - u1_k)) cos(2 pi u2_k)
  *     (Box-Muller), u1, u2 the caller's uniforms in [0, 1) for this step;
+ *   Thompson sampling with the Beta posterior's moments (rewards in [0, 1]; a
+ *     uniform prior, so after N_k rewards summing to R_k the posterior is
+ *     Beta(R_k + 1, N_k - R_k + 1)): a normal draw with its mean and variance,
+ *     argmax_k m_k + z_k sqrt(m_k (1 - m_k) / (N_k + 3)), m_k = (R_k + 1)/(N_k + 2);
  * ties go to the smaller k.  (3) arm = the chosen k.
  */
-enum { BANDIT_UCB1 = 0, BANDIT_THOMPSON = 1 };
+enum { BANDIT_UCB1 = 0, BANDIT_THOMPSON = 1, BANDIT_THOMPSON_BETA = 2 };
 
 int sv_oracle_bandit_step(const int32_t* n_accepted, int B, int gamma, double* t, int32_t* arm, double* N,
                           double* R, int K, int policy, const float* u1, const float* u2)
@@ -522,7 +526,12 @@ int sv_oracle_bandit_step(const int32_t* n_accepted, int B, int gamma, double* t
                 score = R[k] / N[k] + sqrt(2.0 * log(*t) / N[k]);
             } else {
                 const double z = sqrt(-2.0 * log(1.0 - (double)u1[k])) * cos(2.0 * M_PI * (double)u2[k]);
-                score = R[k] / N[k] + z / sqrt(N[k] + 1.0);
+                if (policy == BANDIT_THOMPSON_BETA) {
+                    const double m = (R[k] + 1.0) / (N[k] + 2.0);
+                    score = m + z * sqrt(m * (1.0 - m) / (N[k] + 3.0));
+                } else {
+                    score = R[k] / N[k] + z / sqrt(N[k] + 1.0);
+                }
             }
             if (score > best) { best = score; pick = k; }
         }

@@ -10,7 +10,7 @@ import math
 
 import numpy as np
 
-UCB1, THOMPSON = 0, 1
+UCB1, THOMPSON, THOMPSON_BETA = 0, 1, 2
 
 
 def check_reward_is_accepted_fraction(make):
@@ -131,9 +131,45 @@ def check_thompson_choice_frequency(make):
     assert abs(hits / n - p) < 5 * se, (hits / n, p)
 
 
+def check_thompson_beta_moments(make):
+    """Thompson sampling with the Beta posterior's moments.  After rewards (1, 0) on
+    arm 0 and 0 on arm 1: N = (2, 1), R = (1, 0), so the posteriors are Beta(2, 2)
+    and Beta(1, 2): means (1/2, 1/3), variances (1/20, 1/18).  With z0 = -0.8
+    (u1 = 1 - e^-0.32, u2 = 1/2) and z1 = 0 (u2 = 1/4): theta = (1/2 - 0.8 sqrt(1/20),
+    1/3) = (0.3211, 0.3333) -> arm 1 (the prior's mean: with R/N arm 1 would score 0).
+    Over 20,000 draws arm 1 is chosen with probability Phi((1/3 - 1/2) /
+    sqrt(1/20 + 1/18)) = 0.304 (within 5 standard errors)."""
+    def prepared():
+        b = make(2, THOMPSON_BETA)
+        for x in ([], [1], [0], [0]):
+            b.step(x, 1, [0.5, 0.5], [0.0, 0.0])
+        return b
+    b = prepared()
+    assert b.N.tolist() == [2.0, 1.0] and b.R.tolist() == [1.0, 0.0], (b.N, b.R)
+    u1 = 1.0 - math.exp(-0.32)
+    assert b.step([], 1, [u1, 0.5], [0.5, 0.25]) == 1
+    rng = np.random.default_rng(9)
+    n, hits = 20_000, 0
+    for _ in range(n):
+        hits += b.step([], 1, rng.random(2), rng.random(2)) == 1
+    p = 0.5 * math.erfc((0.5 - 1.0 / 3.0) / math.sqrt(1.0 / 20.0 + 1.0 / 18.0) / math.sqrt(2.0))
+    se = math.sqrt(p * (1 - p) / n)
+    assert abs(hits / n - p) < 5 * se, (hits / n, p)
+
+
+def check_thompson_beta_regret(make):
+    """The Beta-moment policy on T = 10,000 rounds of K = 3 Bernoulli arms (means
+    (0.8, 0.6, 0.3)): mean regret over 6 runs below the Gaussian 1/(N+1) policy's
+    and below 40 (the pages report 18.9 for their Thompson sampling)."""
+    mu, T = (0.8, 0.6, 0.3), 10_000
+    beta = np.mean([_simulate(make, THOMPSON_BETA, mu, T, 300 + s) for s in range(6)])
+    gauss = np.mean([_simulate(make, THOMPSON, mu, T, 300 + s) for s in range(6)])
+    assert beta < gauss and beta < 40.0, (beta, gauss)
+
+
 ALL_BANDIT_CHECKS = [check_reward_is_accepted_fraction, check_ucb1_hand_steps, check_ties_and_unrewarded_first,
                      check_thompson_hand_steps, check_thompson_draw, check_thompson_choice_frequency,
-                     check_regret_within_ucb1_bound]
+                     check_thompson_beta_moments, check_regret_within_ucb1_bound, check_thompson_beta_regret]
 
 
 # ---------------------------------------------------------------------------

@@ -73,6 +73,9 @@ BANDIT_MUTANTS = {
                                   "if (score >= best) { best = score; pick = k; }"),
     "bandit_no_exploration_first": ("if (N[k] == 0.0) { pick = k; break; }", ";"),
     "bandit_thompson_narrow": ("score = R[k] / N[k] + z / sqrt(N[k] + 1.0);", "score = R[k] / N[k] + z / (N[k] + 1.0);"),
+    "bandit_beta_no_prior": ("const double m = (R[k] + 1.0) / (N[k] + 2.0);", "const double m = R[k] / N[k];"),
+    "bandit_beta_variance_n1": ("score = m + z * sqrt(m * (1.0 - m) / (N[k] + 3.0));",
+                                "score = m + z * sqrt(m * (1.0 - m) / (N[k] + 1.0));"),
     "bandit_reward_to_arm0": ("N[*arm] += 1.0;\n        R[*arm] += reward;", "N[*arm] += 1.0;\n        R[0] += reward;"),
 }
 
