@@ -416,7 +416,8 @@ def bandit_row_line(w, dev, lib, binding, cpu_seconds=2.0):
     mud = torch.tensor(mu, dtype=torch.float64, device=dev)
     sim = {"mu": list(mu), "T": BANDIT_T, "runs": BANDIT_RUNS, "ucb1_bound": bound,
            "pages": {"ucb1_regret": 100.2, "ucb1_bound": 526, "thompson_regret": 18.9}}
-    for policy, pname in ((binding.BANDIT_UCB1, "ucb1"), (binding.BANDIT_THOMPSON, "thompson")):
+    for policy, pname in ((binding.BANDIT_UCB1, "ucb1"), (binding.BANDIT_THOMPSON, "thompson"),
+                          (binding.BANDIT_THOMPSON_BETA, "thompson_beta")):
         binding.bandit_simulate(mud, BANDIT_T, policy, Ud)  # warm
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()

@@ -273,6 +273,7 @@ sv_status spec_verify_cache_lookup(const int32_t* out_tokens, const int32_t* out
 #define SV_MAX_ARMS 16
 #define SV_BANDIT_UCB1 0
 #define SV_BANDIT_THOMPSON 1
+#define SV_BANDIT_THOMPSON_BETA 2
 
 /* Bytes of one bandit's state, 8 * (2 + 2K); 0 for K outside [1, SV_MAX_ARMS]. */
 size_t spec_verify_bandit_state_size(int K);
@@ -294,13 +295,16 @@ sv_status spec_verify_bandit_init(double* state, int K, struct CUstream_st* stre
  *        SV_BANDIT_THOMPSON, Gaussian posteriors (Agrawal and Goyal, 2013):
  *            R_k/N_k + z_k / sqrt(N_k + 1),
  *            z_k = sqrt(-2 ln(1 - u1[k])) cos(2 pi u2[k])   (Box-Muller);
+ *        SV_BANDIT_THOMPSON_BETA, a normal draw with the moments of the Beta
+ *            posterior Beta(R_k + 1, N_k - R_k + 1) (uniform prior):
+ *            m_k + z_k sqrt(m_k (1 - m_k) / (N_k + 3)),  m_k = (R_k + 1)/(N_k + 2);
  *      a score that is NaN or -inf never wins; when none wins the arm is -1 and
  *      the next step rewards nothing.
  *  (3) state[1] and *out_arm (if not null) = that arm.
  *
  *   n_accepted  [B] int32 (spec_verify's out_n_accepted); B = 0 rewards nothing
- *   u1, u2      [K] float in [0, 1), this step's uniforms; read for Thompson
- *               sampling only (may be null for UCB1)
+ *   u1, u2      [K] float in [0, 1), this step's uniforms; read for the two
+ *               Thompson policies only (may be null for UCB1)
  *   state       as above;  out_arm  optional [1] int32
  * All pointers are device memory.  The kernel waits (programmatic dependent
  * launch) for the work before it on the stream, so it can follow spec_verify

@@ -28,7 +28,7 @@ EXPORTED = ("spec_verify", "spec_verify_workspace_size", "spec_verify_workspace_
             "spec_verify_lowrank_head")
 MAX_TOPF = 32
 MAX_ARMS = 16
-BANDIT_UCB1, BANDIT_THOMPSON = 0, 1
+BANDIT_UCB1, BANDIT_THOMPSON, BANDIT_THOMPSON_BETA = 0, 1, 2
 MAX_TREE_NODES = 64
 ROW_BAD_TREE = 32
 

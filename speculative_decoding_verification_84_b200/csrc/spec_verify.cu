@@ -649,8 +649,8 @@ extern "C" sv_status spec_verify_bandit_step(const int32_t* n_accepted, int B, i
                                              int32_t* out_arm, struct CUstream_st* stream)
 {
     if (B < 0 || gamma < 1 || K < 1 || K > SV_MAX_ARMS || !state || (B > 0 && !n_accepted) ||
-        (policy != SV_BANDIT_UCB1 && policy != SV_BANDIT_THOMPSON) ||
-        (policy == SV_BANDIT_THOMPSON && (!u1 || !u2)))
+        (policy != SV_BANDIT_UCB1 && policy != SV_BANDIT_THOMPSON && policy != SV_BANDIT_THOMPSON_BETA) ||
+        (policy != SV_BANDIT_UCB1 && (!u1 || !u2)))
         return SV_ERR_INVALID_ARG;
     if (!aligned(n_accepted, 4) || !aligned(u1, 4) || !aligned(u2, 4) || !aligned(state, 8) || !aligned(out_arm, 4))
         return SV_ERR_MISALIGNED;
@@ -673,7 +673,8 @@ extern "C" sv_status spec_verify_bandit_simulate(const double* mu, int K, int T,
                                                  struct CUstream_st* stream)
 {
     if (!mu || K < 1 || K > SV_MAX_ARMS || T < 0 || runs < 0 ||
-        (policy != SV_BANDIT_UCB1 && policy != SV_BANDIT_THOMPSON) || (runs > 0 && (!uniforms || !out_regret)))
+        (policy != SV_BANDIT_UCB1 && policy != SV_BANDIT_THOMPSON && policy != SV_BANDIT_THOMPSON_BETA) ||
+        (runs > 0 && (!uniforms || !out_regret)))
         return SV_ERR_INVALID_ARG;
     if (!aligned(mu, 8) || !aligned(uniforms, 4) || !aligned(out_regret, 8) || !aligned(out_state, 8))
         return SV_ERR_MISALIGNED;

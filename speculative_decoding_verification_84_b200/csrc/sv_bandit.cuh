@@ -14,6 +14,9 @@
 //   Gaussian Thompson sampling (Agrawal and Goyal, 2013):
 //       R_k/N_k + z_k / sqrt(N_k + 1),  z_k = sqrt(-2 ln(1 - u1_k)) cos(2 pi u2_k)
 //       (Box-Muller on the caller's uniforms),
+//   Thompson sampling with the Beta posterior's moments (uniform prior, rewards
+//       in [0, 1]: Beta(R_k + 1, N_k - R_k + 1)):
+//       m_k + z_k sqrt(m_k (1 - m_k) / (N_k + 3)),  m_k = (R_k + 1) / (N_k + 2),
 // the smaller k on ties; a score that is NaN or -inf never wins (arm -1 when no
 // score does, and the next step then rewards nothing).
 //
@@ -48,7 +51,13 @@ __device__ __forceinline__ int bandit_choose(int K, int policy, double t, double
             score = Rk / Nk + sqrt(2.0 * log(t) / Nk);
         } else {
             const double z = sqrt(-2.0 * log(1.0 - (double)u1k)) * cos(2.0 * kBanditPi * (double)u2k);
-            score = Rk / Nk + z / sqrt(Nk + 1.0);
+            if (policy == 2) {
+                const double m = (Rk + 1.0) / (Nk + 2.0);
+                // multiply and add rounded apart (no fused multiply-add), as written
+                score = __dadd_rn(m, __dmul_rn(z, sqrt(__dmul_rn(m, 1.0 - m) / (Nk + 3.0))));
+            } else {
+                score = Rk / Nk + z / sqrt(Nk + 1.0);
+            }
         }
     }
     bool valid = score > -INFINITY;  // false for NaN
@@ -103,8 +112,8 @@ sv_bandit_step(const int32_t* __restrict__ n_accepted, int B, int gamma, int pol
     double Nk = mine ? state[2 + lane] : 0.0;
     double Rk = mine ? state[2 + K + lane] : 0.0;
     if (B > 0) bandit_reward(arm, K, (double)acc / ((double)B * (double)gamma), t, Nk, Rk);
-    const float u1k = (mine && policy == 1) ? u1[lane] : 0.0f;
-    const float u2k = (mine && policy == 1) ? u2[lane] : 0.0f;
+    const float u1k = (mine && policy != 0) ? u1[lane] : 0.0f;
+    const float u2k = (mine && policy != 0) ? u2[lane] : 0.0f;
     const int pick = bandit_choose(K, policy, t, Nk, Rk, u1k, u2k);
     if (mine) {
         state[2 + lane] = Nk;

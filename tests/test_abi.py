@@ -114,7 +114,7 @@ def test_bandit_host_validation(lib):
     assert lib.spec_verify_bandit_init(good, 17, None) == 1
     assert lib.spec_verify_bandit_init(vp((1 << 20) + 4), 3, None) == 3
     step = [good, 4, 5, 0, None, None, good, 3, None, None]
-    bad = list(step); bad[3] = 2                 # unknown policy
+    bad = list(step); bad[3] = 3                 # unknown policy
     assert lib.spec_verify_bandit_step(*bad) == 1
     bad = list(step); bad[3] = 1                 # Thompson sampling without uniforms
     assert lib.spec_verify_bandit_step(*bad) == 1

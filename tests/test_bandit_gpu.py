@@ -25,7 +25,7 @@ def _state_of(b: "oracle.Bandit"):
     return [float(b.t[0]), float(b.arm[0]), *b.N.tolist(), *b.R.tolist()]
 
 
-@pytest.mark.parametrize("policy", [binding.BANDIT_UCB1, binding.BANDIT_THOMPSON])
+@pytest.mark.parametrize("policy", [binding.BANDIT_UCB1, binding.BANDIT_THOMPSON, binding.BANDIT_THOMPSON_BETA])
 @pytest.mark.parametrize("K", [1, 3, 16])
 def test_step_matches_oracle_every_step(policy, K):
     """400 steps of random batches (B from 0 to 3000, gamma 1-8, some steps with an
@@ -85,7 +85,7 @@ def test_fed_by_spec_verify_on_device():
     checks them."""
     K, B, gamma, V = 3, 8, 4, 1000
     noise = (2.5, 0.4, 1.2)  # arm 1 drafts closest to the target
-    for policy in (binding.BANDIT_UCB1, binding.BANDIT_THOMPSON):
+    for policy in (binding.BANDIT_UCB1, binding.BANDIT_THOMPSON, binding.BANDIT_THOMPSON_BETA):
         ref = oracle.Bandit(K, policy)
         state = binding.bandit_state(K, DEV)
         rng = np.random.default_rng(5 + policy)
@@ -121,7 +121,7 @@ def test_fed_by_spec_verify_on_device():
         assert pulls[1] == pulls.max(), pulls  # the best drafts are played most
 
 
-@pytest.mark.parametrize("policy", [binding.BANDIT_UCB1, binding.BANDIT_THOMPSON])
+@pytest.mark.parametrize("policy", [binding.BANDIT_UCB1, binding.BANDIT_THOMPSON, binding.BANDIT_THOMPSON_BETA])
 @pytest.mark.parametrize("mu,T,runs", [((0.75, 0.6, 0.45), 10_000, 96),
                                        ((0.3, 0.5, 0.52, 0.1, 0.49), 3_001, 33),
                                        ((0.5,), 50, 5),
