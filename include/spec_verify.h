@@ -447,7 +447,10 @@ sv_status spec_verify_lowrank_up(const void* u, const void* w_up, int M, int r, 
                                  void* out_logits, double* out_lse, void* workspace, size_t workspace_bytes,
                                  int32_t* out_error, struct CUstream_st* stream);
 
-/* Both contractions: the head from h to the draft logits (and normalisers). */
+/* Both contractions: the head from h to the draft logits (and normalisers).  The
+ * down contraction's K is split across the SMs when its tiles alone are few (its
+ * fp32 slices, kept in the workspace, are added in slice order and rounded to
+ * bf16 once). */
 sv_status spec_verify_lowrank_head(const void* h, const void* w_down, const void* w_up, int M, int d, int r,
                                    int V, const float* temperature, void* out_logits, double* out_lse,
                                    void* workspace, size_t workspace_bytes, int32_t* out_error,

@@ -828,9 +828,10 @@ bool lr_map(CUtensorMap* m, const void* base, long long rows, long long K, int b
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// splits > 1 (no normaliser) needs split_ws: splits * M * N floats.
 template <int BN>
 cudaError_t lr_launch(const void* A, const void* B, int M, int N, int K, void* out, float4* part,
-                      const float* temperature, int* err, cudaStream_t st)
+                      const float* temperature, int* err, cudaStream_t st, int splits = 1, float* split_ws = nullptr)
 {
     CUtensorMap ta, tb, tc;
     if (!lr_map(&ta, A, M, K, sv::kLrBM) || !lr_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
@@ -864,7 +865,9 @@ cudaError_t lr_launch(const void* A, const void* B, int M, int N, int K, void* o
     // A resident: its K blocks plus at least 3 stages of B fit, and every row tile
     // gets at least one CTA
     g.tma_store = tma_store ? 1 : 0;
-    g.a_resident = (kbs <= sv::kLrMaxResidentKb && kbs * a_bytes + 3 * b_bytes <= budget && g.m_tiles <= sms) ? 1 : 0;
+    g.splits = splits;
+    g.part_out = split_ws;
+    g.a_resident = (splits == 1 && kbs <= sv::kLrMaxResidentKb && kbs * a_bytes + 3 * b_bytes <= budget && g.m_tiles <= sms) ? 1 : 0;
     const long long stage = g.a_resident ? b_bytes : a_bytes + b_bytes;
     const long long room = budget - (g.a_resident ? kbs * a_bytes : 0);
     g.stages = (int)std::min<long long>(sv::kLrMaxStages, room / stage);
@@ -873,11 +876,17 @@ cudaError_t lr_launch(const void* A, const void* B, int M, int N, int K, void* o
         const long long slots = std::min<long long>(sms / g.m_tiles, g.n_tiles);
         grid = slots * g.m_tiles;
     } else {
-        grid = std::min<long long>(tiles, sms);  // one CTA per SM (shared memory)
+        grid = std::min<long long>(tiles * splits, sms);  // one CTA per SM (shared memory)
     }
     const long long smem =
         1024 + (g.a_resident ? kbs * a_bytes : 0) + g.stages * stage + (tma_store ? sv::kLrStagingBytes : 0);
     sv::sv_lr_gemm<BN><<<(unsigned)grid, sv::kLrThreads, (size_t)smem, st>>>(ta, tb, tc, g);
+    if (splits > 1) {
+        if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+        const long long total = (long long)M * N;
+        const unsigned blocks = (unsigned)std::min<long long>(cdiv(total, 256), 4LL * sms);
+        sv::sv_lr_splitk_sum<<<blocks, 256, 0, st>>>(split_ws, splits, M, N, static_cast<__nv_bfloat16*>(out));
+    }
     return cudaGetLastError();
 }
 
@@ -890,8 +899,21 @@ bool lr_shape_ok(int M, int d, int r, int V)
 
 constexpr int kLrUpBN = 256;
 constexpr int kLrDownBN = 32;
+constexpr int kLrMaxSplits = 8;
+
+// K slices for the down contraction inside the head: enough CTAs to fill the SMs
+// when its tiles alone are few, each slice at least 4 K blocks.
+int lr_down_splits(int M, int d, int r)
+{
+    const long long tiles = cdiv(M, sv::kLrBM) * cdiv(r, kLrDownBN);
+    const long long kbs = cdiv(d, sv::kLrBK);
+    long long s = std::max<long long>(1, device_sm_count() / std::max<long long>(tiles, 1));
+    s = std::min<long long>(s, std::min<long long>(kLrMaxSplits, kbs / 4));
+    return (int)std::max<long long>(s, 1);
+}
 
 size_t lr_u_bytes(int M, int r) { return ((size_t)M * r * 2 + 1023) / 1024 * 1024; }
+size_t lr_split_bytes(int M, int r) { return ((size_t)kLrMaxSplits * M * r * 4 + 1023) / 1024 * 1024; }
 size_t lr_part_bytes(int M, int V) { return (size_t)M * (size_t)cdiv(V, kLrUpBN) * sv::kLrGroups * sizeof(float4); }
 
 }  // namespace
@@ -899,7 +921,7 @@ size_t lr_part_bytes(int M, int V) { return (size_t)M * (size_t)cdiv(V, kLrUpBN)
 extern "C" size_t spec_verify_lowrank_workspace_size(int M, int r, int V)
 {
     if (M < 1 || r < 8 || (r % 8) != 0 || V < 1 || V > SV_MAX_V) return 0;
-    return lr_u_bytes(M, r) + lr_part_bytes(M, V);
+    return lr_u_bytes(M, r) + lr_split_bytes(M, r) + lr_part_bytes(M, V);
 }
 
 extern "C" sv_status spec_verify_lowrank_down(const void* h, const void* w_down, int M, int d, int r, void* out_u,
@@ -948,9 +970,14 @@ extern "C" sv_status spec_verify_lowrank_head(const void* h, const void* w_down,
     if (!aligned(workspace, 256)) return SV_ERR_MISALIGNED;
     if (workspace_bytes < spec_verify_lowrank_workspace_size(M, r, V)) return SV_ERR_WORKSPACE_TOO_SMALL;
     void* u = workspace;
-    void* rest = static_cast<unsigned char*>(workspace) + lr_u_bytes(M, r);
-    const sv_status s = spec_verify_lowrank_down(h, w_down, M, d, r, u, out_error, stream);
-    if (s != SV_OK) return s;
-    return spec_verify_lowrank_up(u, w_up, M, r, V, temperature, out_logits, out_lse, rest,
-                                  workspace_bytes - lr_u_bytes(M, r), out_error, stream);
+    float* split_ws = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + lr_u_bytes(M, r));
+    const size_t head = lr_u_bytes(M, r) + lr_split_bytes(M, r);
+    void* rest = static_cast<unsigned char*>(workspace) + head;
+    if (!aligned(h, 16) || !aligned(w_down, 16)) return SV_ERR_MISALIGNED;
+    // the down contraction, its K split across the SMs (its tiles alone are few)
+    const cudaError_t e = lr_launch<kLrDownBN>(h, w_down, M, r, d, u, nullptr, nullptr, out_error,
+                                               (cudaStream_t)stream, lr_down_splits(M, d, r), split_ws);
+    if (e != cudaSuccess) return e == cudaErrorInvalidValue ? SV_ERR_INVALID_ARG : SV_ERR_CUDA;
+    return spec_verify_lowrank_up(u, w_up, M, r, V, temperature, out_logits, out_lse, rest, workspace_bytes - head,
+                                  out_error, stream);
 }

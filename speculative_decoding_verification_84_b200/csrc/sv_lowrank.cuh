@@ -58,6 +58,8 @@ struct LrArgs {
     int stages;                // ring depth
     int a_resident;            // the CTA's A tile (all of K) is loaded once and kept
     int tma_store;             // out written by TMA stores of 32 x 32 chunks staged in shared memory
+    int splits;                // K split this many ways (no A residency, no normaliser): each
+    float* part_out;           // slice writes fp32 [splits][M][N] here, summed by sv_lr_splitk_sum
 };
 
 constexpr int kLrChunkBytes = 32 * 32 * 2;                      // one 32-row x 32-column bf16 chunk
@@ -186,8 +188,9 @@ __device__ __forceinline__ void lr_arrive(uint64_t* bar)
 // CTAs of one slot run the same column tile at about the same time, so its W
 // rows come from HBM once); otherwise tiles c, c + gridDim.x, ... with the row
 // tile fastest.
-__device__ __forceinline__ bool lr_tile(const LrArgs& g, int k, int* m, int* n)
+__device__ __forceinline__ bool lr_tile(const LrArgs& g, int k, int* m, int* n, int* ks)
 {
+    *ks = 0;
     if (g.a_resident) {
         const int nslots = (int)gridDim.x / g.m_tiles;
         *m = (int)blockIdx.x % g.m_tiles;
@@ -195,10 +198,20 @@ __device__ __forceinline__ bool lr_tile(const LrArgs& g, int k, int* m, int* n)
         return *n < g.n_tiles;
     }
     const long long t = (long long)blockIdx.x + (long long)k * gridDim.x;
-    if (t >= (long long)g.m_tiles * g.n_tiles) return false;
+    if (t >= (long long)g.m_tiles * g.n_tiles * g.splits) return false;
     *m = (int)(t % g.m_tiles);
-    *n = (int)(t / g.m_tiles);
+    const long long rest = t / g.m_tiles;
+    *n = (int)(rest % g.n_tiles);
+    *ks = (int)(rest / g.n_tiles);
     return true;
+}
+
+// K blocks [kb0, kb1) of slice ks.
+__device__ __forceinline__ void lr_kslice(const LrArgs& g, int kbs, int ks, int* kb0, int* kb1)
+{
+    const int per = (kbs + g.splits - 1) / g.splits;
+    *kb0 = min(kbs, ks * per);
+    *kb1 = min(kbs, *kb0 + per);
 }
 
 // Persistent, one CTA per SM; the accumulator is double-buffered in TMEM (2 x BN
@@ -258,16 +271,18 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     int issued = 0, a_issued = 0;
     if (warp == 0 && lane == 0) {
         // ---- producer: one global count of stages across the CTA's tiles
-        int m0, n0;
-        if (res && lr_tile(g, 0, &m0, &n0)) {
+        int m0, n0, k0;
+        if (res && lr_tile(g, 0, &m0, &n0, &k0)) {
             lr_expect_tx(&afull, (unsigned)(kbs * A_BYTES));
             for (int kb = 0; kb < kbs; ++kb) lr_tma_2d(sm + kb * A_BYTES, &ta, &afull, kb * kLrBK, m0 * kLrBM);
             a_issued = 1;
         }
-        int it = 0, m, n;
+        int it = 0, m, n, ks;
         bool ok = true;
-        for (int k = 0; ok && lr_tile(g, k, &m, &n); ++k) {
-            for (int kb = 0; kb < kbs; ++kb, ++it) {
+        for (int k = 0; ok && lr_tile(g, k, &m, &n, &ks); ++k) {
+            int kb0, kb1;
+            lr_kslice(g, kbs, ks, &kb0, &kb1);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % S;
                 const unsigned ph = (unsigned)(it / S);
                 if (it >= S && !lr_wait(&empty[s], (ph - 1u) & 1u, abort, g.err)) { ok = false; break; }
@@ -281,18 +296,20 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer
         constexpr uint32_t idesc = lr_idesc<BN>();
-        int it = 0, i = 0, m, n;
+        int it = 0, i = 0, m, n, ks;
         bool ok = true;
-        if (res && lr_tile(g, 0, &m, &n)) {
+        if (res && lr_tile(g, 0, &m, &n, &ks)) {
             ok = lr_wait(&afull, 0u, abort, g.err);
             s_a_done = ok ? 1 : 0;
         }
-        for (; ok && lr_tile(g, i, &m, &n); ++i) {
+        for (; ok && lr_tile(g, i, &m, &n, &ks); ++i) {
             const int b = i & 1, use = i >> 1;
             if (use >= 1 && !lr_wait(&tempty[b], (unsigned)(use - 1) & 1u, abort, g.err)) break;
             lr_fence_after();
             const uint32_t d = tmem + (uint32_t)(b * BN);
-            for (int kb = 0; kb < kbs; ++kb, ++it) {
+            int kb0, kb1;
+            lr_kslice(g, kbs, ks, &kb0, &kb1);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % S;
                 const unsigned ph = (unsigned)(it / S);
                 if (!lr_wait(&full[s], ph & 1u, abort, g.err)) { ok = false; break; }
@@ -302,7 +319,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
                 const uint32_t b0 = res ? st : st + A_BYTES;
 #pragma unroll
                 for (int j = 0; j < kLrBK / 16; ++j)  // K = 16 per MMA: 32 bytes along the swizzled row
-                    lr_mma(d, lr_desc(a0 + 32 * j), lr_desc(b0 + 32 * j), idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                    lr_mma(d, lr_desc(a0 + 32 * j), lr_desc(b0 + 32 * j), idesc, (kb > kb0 || j > 0) ? 1u : 0u);
                 lr_commit(&empty[s]);
                 s_consumed = it + 1;
             }
@@ -319,8 +336,8 @@ __global__ void __launch_bounds__(kLrThreads, 1)
         const bool lse = g.part != nullptr;
         unsigned char* stg = staging + (warp - 4) * 2 * kLrChunkBytes;
         int chunks = 0;  // chunks this warp has staged (the buffer alternates)
-        int i = 0, m_tile, n_tile;
-        for (; lr_tile(g, i, &m_tile, &n_tile); ++i) {
+        int i = 0, m_tile, n_tile, ks;
+        for (; lr_tile(g, i, &m_tile, &n_tile, &ks); ++i) {
             const int b = i & 1, use = i >> 1;
             const int row = m_tile * kLrBM + 32 * q + lane;
             const bool row_ok = row < g.M;
@@ -355,6 +372,22 @@ __global__ void __launch_bounds__(kLrThreads, 1)
                     if (lane == 0) lr_arrive(&tempty[b]);
                 }
                 const int n0 = n_tile * BN + grp * QCOLS + c;
+                if (g.splits > 1) {
+                    // a K slice: the raw fp32 sums, for sv_lr_splitk_sum
+                    if (row_ok) {
+                        float* dst = g.part_out + ((size_t)ks * g.M + row) * g.N + n0;
+                        if (n0 + 32 <= g.N && (g.N & 3) == 0) {
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                reinterpret_cast<uint4*>(dst)[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)  // unrolled: r stays in registers
+                                if (n0 + k < g.N) dst[k] = __uint_as_float(r[k]);
+                        }
+                    }
+                    continue;
+                }
                 float x[32];
                 uint32_t packed[16];
 #pragma unroll
@@ -388,11 +421,11 @@ __global__ void __launch_bounds__(kLrThreads, 1)
                             reinterpret_cast<uint4*>(dst)[v] =
                                 make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                     } else {
-                        for (int k = 0; k < 32 && n0 + k < g.N; ++k) {
-                            const uint32_t w = packed[k / 2];
-                            reinterpret_cast<unsigned short*>(dst)[k] =
-                                (unsigned short)((k & 1) ? (w >> 16) : (w & 0xffffu));
-                        }
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)  // unrolled: packed stays in registers
+                            if (n0 + k < g.N)
+                                reinterpret_cast<unsigned short*>(dst)[k] =
+                                    (unsigned short)((k & 1) ? (packed[k / 2] >> 16) : (packed[k / 2] & 0xffffu));
                     }
                 }
                 if (lse_row) {
@@ -436,6 +469,19 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     if (warp == 2) {
         lr_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
+    }
+}
+
+// out [M][N] = bf16 of the sum of the K slices' fp32 partials, slice 0 first.
+__global__ void sv_lr_splitk_sum(const float* __restrict__ part, int splits, int M, int N,
+                                 __nv_bfloat16* __restrict__ out)
+{
+    const long long total = (long long)M * N;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        float acc = part[i];
+        for (int s = 1; s < splits; ++s) acc += part[(long long)s * total + i];
+        out[i] = __float2bfloat16_rn(acc);
     }
 }
 
