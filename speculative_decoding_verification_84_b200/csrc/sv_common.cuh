@@ -218,6 +218,20 @@ __device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigne
     return d;
 }
 
+__device__ __forceinline__ unsigned long long sub2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // lse_group with the exponent arguments and the accumulations done on packed
 // pairs.  Element e of a vector still goes to acc[e & 7] in the same order, and
 // every operation rounds as in lse_group, so the two give identical bits; this

@@ -430,19 +430,32 @@ __global__ void __launch_bounds__(kLrThreads, 1)
                 }
                 if (lse_row) {
                     // one maximum and at most one rescale per 32 columns, then 32
-                    // independent terms into 8 accumulators
-                    float vm = -INFINITY;
+                    // independent terms on packed fp32 pairs (each term rounds as
+                    // scaled_exp's), columns past N only in the last column tile
+                    if (n0 + 32 > g.N) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        if (n0 + k >= g.N) x[k] = -INFINITY;  // columns past N take no part
-                        vm = fmaxf(vm, x[k]);
+                        for (int k = 0; k < 32; ++k)
+                            if (n0 + k >= g.N) x[k] = -INFINITY;
                     }
+                    float vm = x[0];
+#pragma unroll
+                    for (int k = 1; k < 32; ++k) vm = fmaxf(vm, x[k]);
                     lse_rebase(L, vm, khi);
+                    const unsigned long long KH = pack2(khi, khi), KL = pack2(klo, klo), NM = pack2(-L.mk, -L.mk);
+                    unsigned long long acc2[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc2[e] = pack2(0.f, 0.f);
+#pragma unroll
+                    for (int k = 0; k < 32; k += 2) {
+                        const unsigned long long x2 = pack2(x[k], x[k + 1]);
+                        const unsigned long long y2 = fma2(x2, KL, fma2(x2, KH, NM));
+                        float y0, y1;
+                        unpack2(y2, y0, y1);
+                        acc2[(k >> 1) & 3] = add2(acc2[(k >> 1) & 3], pack2(ex2(y0), ex2(y1)));
+                    }
                     float acc[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) acc[k & 7] += scaled_exp(x[k], khi, klo, L.mk);
+                    for (int e = 0; e < 4; ++e) unpack2(acc2[e], acc[2 * e], acc[2 * e + 1]);
                     L.s += tree8(acc);
                 }
             }

@@ -166,6 +166,50 @@ __device__ __forceinline__ float tree_weight(const TreeRow& r, const float* inv_
     return resid ? fmaxf(0.f, P - q) : P;
 }
 
+// tree_weight for elements (0, 1) of a pair on packed fp32 pairs: every
+// operation rounds as its scalar form in tree_weight, so both give the same bits.
+__device__ __forceinline__ void tree_weight2(const TreeRow& r, const float* inv_S, int level, bool resid, float lt0,
+                                             float lt1, float ld0, float ld1, float& w0, float& w1)
+{
+    const unsigned long long KH = pack2(r.khi, r.khi), KL = pack2(r.klo, r.klo);
+    const unsigned long long xt = pack2(lt0, lt1);
+    float a0, a1;
+    unpack2(fma2(xt, KL, fma2(xt, KH, pack2(-r.mk_t, -r.mk_t))), a0, a1);
+    unsigned long long P = mul2(pack2(ex2(a0), ex2(a1)), pack2(r.inv_t, r.inv_t));
+    if (level == 0 && !resid) {
+        unpack2(P, w0, w1);
+        return;
+    }
+    const unsigned long long xd = pack2(ld0, ld1);
+    float b0, b1;
+    unpack2(fma2(xd, KL, fma2(xd, KH, pack2(-r.mk_d, -r.mk_d))), b0, b1);
+    const unsigned long long Q = mul2(pack2(ex2(b0), ex2(b1)), pack2(r.inv_d, r.inv_d));
+    for (int k = 0; k < level; ++k) {
+        float d0, d1;
+        unpack2(sub2(P, Q), d0, d1);
+        P = mul2(pack2(fmaxf(0.f, d0), fmaxf(0.f, d1)), pack2(inv_S[k], inv_S[k]));
+    }
+    if (resid) {
+        float d0, d1;
+        unpack2(sub2(P, Q), d0, d1);
+        w0 = fmaxf(0.f, d0);
+        w1 = fmaxf(0.f, d1);
+    } else {
+        unpack2(P, w0, w1);
+    }
+}
+
+// The weights of one 16-byte group (VEC elements, padded with zeros to 8).
+template <int VEC>
+__device__ __forceinline__ void tree_group_weights(const TreeRow& r, const float* inv_S, int level, bool resid,
+                                                   const float* xt, const float* xd, float (&wv)[8])
+{
+#pragma unroll
+    for (int e = 0; e < VEC; e += 2) tree_weight2(r, inv_S, level, resid, xt[e], xt[e + 1], xd[e], xd[e + 1], wv[e], wv[e + 1]);
+#pragma unroll
+    for (int e = VEC; e < 8; ++e) wv[e] = 0.f;
+}
+
 struct TreeSmem {
     TreeSlot x[2][kTreeMaxCluster];   // exchange buffers, alternating
     Lse wl[2][kTreeWarps];            // per-warp row states
@@ -394,10 +438,8 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
             const double lp = level == 0 ? (double)sm.lt[k] / Td - a2t * kLn2
                                          : log((double)tree_weight(rw, sm.inv_S, level, false, sm.lt[k], sm.ld[k]));
             if (log((double)a.u_accept[(size_t)b * N + i]) < lp - lq) { next = i; break; }
-            // rejected: the mass of max(0, P - q) (and its last positive token, for
-            // a draw that may reuse these sums)
+            // rejected: the mass of max(0, P - q)
             double part = 0.0;
-            int last = -1;
             for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
                 uint4 rt[kTreeBatch], rd[kTreeBatch];
 #pragma unroll
@@ -412,26 +454,18 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
                         float xt[VEC], xd[VEC], wv[8];
                         unpack<ESZ>(rt[u], xt);
                         unpack<ESZ>(rd[u], xd);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            wv[e] = e < VEC ? tree_weight(rw, sm.inv_S, level, true, xt[e], xd[e]) : 0.f;
-                            if (e < VEC && wv[e] > 0.f) last = (int)((g0 + 32 * u) * VEC + e);
-                        }
+                        tree_group_weights<VEC>(rw, sm.inv_S, level, true, xt, xd, wv);
                         part += (double)tree8(wv);
                     }
             }
             part = warp_sum(part);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-            if (lane == 0) { sm.wsum[warp] = part; sm.wlast[warp] = last; }
+            if (lane == 0) sm.wsum[warp] = part;
             __syncthreads();
             if (tid == 0) {
                 double s = 0.0;
-                int l = -1;
-                for (int w = 0; w < kTreeWarps; ++w) { s += sm.wsum[w]; l = max(l, sm.wlast[w]); }
+                for (int w = 0; w < kTreeWarps; ++w) s += sm.wsum[w];
                 TreeSlot t{};
                 t.s[0] = s;
-                t.idx = l;
                 s_mine = t;
             }
             __syncthreads();
@@ -464,7 +498,6 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         int dpar = reuse_par;
         if (dpar < 0) {
             double part = 0.0;
-            int last = -1;
             for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
                 uint4 rt[kTreeBatch], rd[kTreeBatch];
 #pragma unroll
@@ -479,26 +512,18 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
                         float xt[VEC], xd[VEC], wv[8];
                         unpack<ESZ>(rt[u], xt);
                         unpack<ESZ>(rd[u], xd);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            wv[e] = e < VEC ? tree_weight(rw, sm.inv_S, lev, resid, xt[e], xd[e]) : 0.f;
-                            if (e < VEC && wv[e] > 0.f) last = (int)((g0 + 32 * u) * VEC + e);
-                        }
+                        tree_group_weights<VEC>(rw, sm.inv_S, lev, resid, xt, xd, wv);
                         part += (double)tree8(wv);
                     }
             }
             part = warp_sum(part);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-            if (lane == 0) { sm.wsum[warp] = part; sm.wlast[warp] = last; }
+            if (lane == 0) sm.wsum[warp] = part;
             __syncthreads();
             if (tid == 0) {
                 double s = 0.0;
-                int l = -1;
-                for (int w = 0; w < kTreeWarps; ++w) { s += sm.wsum[w]; l = max(l, sm.wlast[w]); }
+                for (int w = 0; w < kTreeWarps; ++w) s += sm.wsum[w];
                 TreeSlot t{};
                 t.s[0] = s;
-                t.idx = l;
                 s_mine = t;
             }
             __syncthreads();
@@ -507,9 +532,30 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
             xpar ^= 1;
         }
         double S = 0.0;
-        int lastpos = -1;
-        for (int q = 0; q < CL; ++q) { S += sm.x[dpar][q].s[0]; lastpos = max(lastpos, sm.x[dpar][q].idx); }
+        for (int q = 0; q < CL; ++q) S += sm.x[dpar][q].s[0];
         const double target = (double)a.u_resample[b] * S;
+        // the last token of this CTA's range with a positive weight (-1 if none):
+        // only for the rare draw that rounding leaves without a crossing
+        auto cta_last_positive = [&]() -> int {
+            int last = -1;
+            for (long long g = lo + lane; g < hi; g += 32) {
+                float xt[VEC], xd[VEC];
+                const uint4 rt = tree_raw<ESZ, VEC16>(trow, g, V);
+                unpack<ESZ>(rt, xt);
+                unpack<ESZ>(resid ? tree_raw<ESZ, VEC16>(drow, g, V) : rt, xd);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    if (tree_weight(rw, sm.inv_S, lev, resid, xt[e], xd[e]) > 0.f) last = (int)(g * VEC + e);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+            if (lane == 0) sm.wlast[warp] = last;
+            __syncthreads();
+            int l = -1;
+            for (int w = 0; w < kTreeWarps; ++w) l = max(l, sm.wlast[w]);
+            __syncthreads();
+            return l;
+        };
         // the CTA whose range holds the crossing
         int rstar = -1;
         double before = 0.0;
@@ -521,8 +567,23 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
                 C += s;
             }
         }
-        extra = lastpos;  // if rounding leaves no crossing: the last token with a positive weight
         writer = rstar >= 0 ? rstar : 0;
+        if (rstar < 0) {
+            // rounding left no crossing: the last token with a positive weight
+            // over the whole row (every CTA of the cluster takes this branch)
+            const int l = cta_last_positive();
+            if (tid == 0) {
+                TreeSlot t{};
+                t.idx = l;
+                s_mine = t;
+            }
+            __syncthreads();
+            tree_exchange(cl, sm, xpar, s_mine, CL, rank);
+            int lastpos = -1;
+            for (int q = 0; q < CL; ++q) lastpos = max(lastpos, sm.x[xpar][q].idx);
+            xpar ^= 1;
+            extra = lastpos;
+        }
         if (rstar == rank) {
             // warp holding the crossing, then its 32-group blocks, lanes and elements
             __shared__ int s_found;
@@ -580,6 +641,7 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
             }
             __syncthreads();
             if (s_found <= -2) extra = -2 - s_found;
+            else extra = cta_last_positive();  // the search lost the crossing to rounding
         }
         break;
     }
