@@ -723,14 +723,24 @@ __global__ void __launch_bounds__(kPruneThreads) sv_tree_prune_rows(PruneArgs a)
     Lse L;
     lse_init(L);
     Amax A{-INFINITY, 0x7fffffff, 0};
-    for (long long g = tid; g < a.G; g += kPruneThreads) {
-        float x[VEC];
-        unpack<ESZ>(tree_raw<ESZ, VEC16>(row, g, a.V), x);
-        if (greedy) {
+    constexpr int kPB = 4;  // groups per thread loaded before any is used
+    for (long long g0 = tid; g0 < a.G; g0 += (long long)kPruneThreads * kPB) {
+        uint4 raw[kPB];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) amax_add(A, x[e], (int)(g * VEC + e));
-        } else {
-            lse_add<VEC>(L, x, khi, klo);
+        for (int u = 0; u < kPB; ++u)
+            if (g0 + (long long)kPruneThreads * u < a.G) raw[u] = tree_raw<ESZ, VEC16>(row, g0 + (long long)kPruneThreads * u, a.V);
+#pragma unroll
+        for (int u = 0; u < kPB; ++u) {
+            const long long g = g0 + (long long)kPruneThreads * u;
+            if (g >= a.G) break;
+            float x[VEC];
+            unpack<ESZ>(raw[u], x);
+            if (greedy) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) amax_add(A, x[e], (int)(g * VEC + e));
+            } else {
+                lse_add<VEC>(L, x, khi, klo);
+            }
         }
     }
     const int nanf = __any_sync(0xffffffffu, L.s != L.s);
