@@ -846,6 +846,25 @@ def run_profile(args):
     from speculative_decoding_verification_84_b200 import binding, build, workloads as W
     build.build()
     lib = binding.load_library()
+    if args.profile == "c3topf":
+        w = W.make_workload("c3")
+        d = binding.to_device(w, "cuda:0")
+        _, _, ln, st = binding.verify(**d, return_log_norm=True, return_row_status=True)
+        F = np.minimum(binding.fanout(0.7, w.gamma, 64), binding.MAX_TOPF).astype(np.int32)
+        for i in range(args.warmup + args.steps):
+            binding.topf(d["target"], d["draft"], d["temperature"], ln, st, F)
+        torch.cuda.synchronize()
+        print(f"c3topf: {args.warmup + args.steps} calls, 1 launch each", flush=True)
+        return 0
+    if args.profile == "bandit":
+        from speculative_decoding_verification_84_b200 import workloads as W2
+        U = torch.from_numpy(W2.bandit_uniforms(BANDIT_RUNS, BANDIT_T, 3, seed=2002)).to("cuda:0")
+        mu = torch.tensor(BANDIT_MU, dtype=torch.float64, device="cuda:0")
+        for i in range(args.warmup + args.steps):
+            binding.bandit_simulate(mu, BANDIT_T, binding.BANDIT_THOMPSON_BETA, U)
+        torch.cuda.synchronize()
+        print(f"bandit: {args.warmup + args.steps} simulations, 1 launch each", flush=True)
+        return 0
     if args.profile == "h3":
         M, d, r, V = LOWRANK_SHAPE
         w = W.make_lowrank(M, d, r, V, seed=2005, T=1.0)
@@ -881,7 +900,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="skip the line's per-workload numbers")
-    ap.add_argument("--profile", choices=list(PER_CONFIG) + ["t3", "h3"], default=None,
+    ap.add_argument("--profile", choices=list(PER_CONFIG) + ["t3", "h3", "c3topf", "bandit"], default=None,
                     help="only make warm-up + K calls of this workload (for a profiler); no JSON line")
     args = ap.parse_args()
     if args.profile:
