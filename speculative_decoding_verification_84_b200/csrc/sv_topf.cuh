@@ -82,10 +82,11 @@ __device__ __forceinline__ unsigned qualifying(const float (&w)[VEC], int i0, fl
     return qm;
 }
 
-// Insert every qualifying candidate of the warp, one per round: the lowest lane
-// that has one offers its first; then every lane re-tests its own against the
-// raised bar.  The rounds are as many as the insertions (the final list does not
-// depend on their order: the ranking is a total order).
+// Offer every qualifying candidate of the warp, one per round: the lowest lane
+// that has one offers its first; the candidate is inserted if it still ranks
+// before the list's last pair (the list may have moved on since the lane's vote),
+// else dropped.  The final list does not depend on the order of the offers: the
+// ranking is a total order.
 template <int VEC>
 __device__ __forceinline__ void list_offer_vec(float& lw, int& lv, float& tw, int& tv, const float (&w)[VEC],
                                                int i0, int F, unsigned qm, int* s_bar)
@@ -102,16 +103,33 @@ __device__ __forceinline__ void list_offer_vec(float& lw, int& lv, float& tw, in
             if (e == e0) cw = w[e];
         cw = __shfl_sync(0xffffffffu, cw, src);
         const int cv = __shfl_sync(0xffffffffu, i0 + e0, src);
-        list_insert(lw, lv, cw, cv, F);
-        tw = __shfl_sync(0xffffffffu, lw, F - 1);
-        tv = __shfl_sync(0xffffffffu, lv, F - 1);
         if (lane == src) qm &= ~(1u << e0);
-        qm &= qualifying<VEC>(w, i0, tw, tv, 0.f);
+        if (ranks_before(cw, cv, tw, tv)) {  // the same in every lane
+            list_insert(lw, lv, cw, cv, F);
+            tw = __shfl_sync(0xffffffffu, lw, F - 1);
+            tv = __shfl_sync(0xffffffffu, lv, F - 1);
+        }
         m = __ballot_sync(0xffffffffu, qm != 0);
     }
     // a full list's last weight bounds the CTA's F-th weight from below: publish it
     // (weights are >= 0, so their bit patterns order as integers)
     if (lane == 0 && tw > 0.f) atomicMax(s_bar, __float_as_int(tw));
+}
+
+// The F-th largest of the warp's 32 values (one per lane), by a bitonic sort in
+// descending order across the lanes.  F <= 32.
+__device__ __forceinline__ float warp_fth_largest(float v, int F)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const float o = __shfl_xor_sync(0xffffffffu, v, j);
+            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+            v = keep_max ? fmaxf(v, o) : fminf(v, o);
+        }
+    return __shfl_sync(0xffffffffu, v, F - 1);
 }
 
 // The weights of row pair (t, d) at element i: max(0, p - q), or p (p_only),
@@ -126,6 +144,29 @@ __device__ __forceinline__ float topf_weight(const TopfScale& z, bool p_only, fl
     if (p_only) return p;
     const float q = ex2(__fmaf_rn(ld, z.klo, __fmaf_rn(ld, z.khi, -z.md))) * z.cd;
     return fmaxf(0.f, p - q);
+}
+
+// topf_weight for elements (0, 1) of a pair on packed fp32 pairs (every
+// operation rounds as in topf_weight, so both give the same bits).
+__device__ __forceinline__ void topf_weight2(const TopfScale& z, bool p_only, float lt0, float lt1, float ld0, float ld1,
+                                             float& w0, float& w1)
+{
+    const unsigned long long KH = pack2(z.khi, z.khi), KL = pack2(z.klo, z.klo);
+    const unsigned long long xt = pack2(lt0, lt1);
+    float a0, a1;
+    unpack2(fma2(xt, KL, fma2(xt, KH, pack2(-z.mt, -z.mt))), a0, a1);
+    const unsigned long long P = mul2(pack2(ex2(a0), ex2(a1)), pack2(z.ct, z.ct));
+    if (p_only) {
+        unpack2(P, w0, w1);
+        return;
+    }
+    const unsigned long long xd = pack2(ld0, ld1);
+    float b0, b1;
+    unpack2(fma2(xd, KL, fma2(xd, KH, pack2(-z.md, -z.md))), b0, b1);
+    float d0, d1;
+    unpack2(sub2(P, mul2(pack2(ex2(b0), ex2(b1)), pack2(z.cd, z.cd))), d0, d1);
+    w0 = fmaxf(0.f, d0);
+    w1 = fmaxf(0.f, d1);
 }
 
 // The sum of a vector's weights, as a short tree (4 or 8 elements).
@@ -149,6 +190,12 @@ __device__ void topf_pass(const TopfArgs& g, const unsigned char* rt, const unsi
     float lw = -1.f, tw = -1.f;
     int lv = 0x7fffffff, tv = 0x7fffffff;
     double ls = 0.0;
+    // a floor under this warp's candidates, from its first vectors: the F-th
+    // largest of the 32 lanes' largest weights.  At least F weights reach it, so no
+    // weight below it is among the CTA's F largest; it spares the rounds that an
+    // empty list would otherwise spend on every positive weight.
+    float floor_w = 0.f;
+    bool seeded = false;
     if (vec) {
         const int nv = V / VEC;
         const int per = (nv + kTopfWarps - 1) / kTopfWarps;
@@ -171,13 +218,26 @@ __device__ void topf_pass(const TopfArgs& g, const unsigned char* rt, const unsi
             unpack<ESZ>(vd[u], xd);
             float w[VEC];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) w[e] = ok ? topf_weight(z, p_only, xt[e], xd[e]) : 0.f;
+            for (int e = 0; e < VEC; e += 2) topf_weight2(z, p_only, xt[e], xt[e + 1], xd[e], xd[e + 1], w[e], w[e + 1]);
+            if (!ok) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) w[e] = 0.f;
+            }
             ls += (double)tree8_any<VEC>(w);
             // one vote per vector; rounds only for the candidates that beat the list
             // and are not below another warp's published F-th weight (F pairs of that
-            // warp outrank them)
-            const float bar = __int_as_float(*reinterpret_cast<volatile int*>(s_bar));
-            list_offer_vec<VEC>(lw, lv, tw, tv, w, q * VEC, F, qualifying<VEC>(w, q * VEC, tw, tv, bar), s_bar);
+            // warp outrank them).  The elements are tested only when the vector's
+            // largest weight could qualify.
+            float vmax = w[0];
+#pragma unroll
+            for (int e = 1; e < VEC; ++e) vmax = fmaxf(vmax, w[e]);
+            if (!seeded) {  // the first vectors (uniform across the warp)
+                floor_w = warp_fth_largest(vmax, F);
+                seeded = true;
+            }
+            const float bar = fmaxf(__int_as_float(*reinterpret_cast<volatile int*>(s_bar)), floor_w);
+            const unsigned qm = (vmax > 0.f && vmax >= bar && vmax >= tw) ? qualifying<VEC>(w, q * VEC, tw, tv, bar) : 0u;
+            list_offer_vec<VEC>(lw, lv, tw, tv, w, q * VEC, F, qm, s_bar);
             }
         }
     } else {
