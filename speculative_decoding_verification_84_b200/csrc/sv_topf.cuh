@@ -17,7 +17,7 @@
 //                    its part of the rows in its lanes (lane i: the i-th best,
 //                    by weight, then smaller token); a candidate that beats lane
 //                    F_n - 1 is inserted by one ballot and one shuffle.  The CTA
-//                    then sorts the warps' 16 x 32 candidates (bitonic, shared
+//                    then sorts the warps' 8 x 32 candidates (bitonic, shared
 //                    memory) and keeps the first F_n.
 //   sv_cache_lookup  one thread per sequence: the slot of outcome n's list that
 //                    holds the extra token spec_verify emitted, else -1.
@@ -27,7 +27,7 @@
 
 namespace sv {
 
-constexpr int kTopfThreads = 512;
+constexpr int kTopfThreads = 256;  // 3 CTAs per SM: 64 x 6 outcomes in one wave on 148 SMs
 constexpr int kTopfWarps = kTopfThreads / 32;
 constexpr int kTopfBatch = 4;  // 16-byte vectors per lane and row loaded before any is used
 
@@ -285,7 +285,7 @@ __device__ void topf_pass(const TopfArgs& g, const unsigned char* rt, const unsi
 }
 
 template <int ESZ>
-__global__ void __launch_bounds__(kTopfThreads, 1) sv_topf(const __grid_constant__ TopfArgs g)
+__global__ void __launch_bounds__(kTopfThreads, 3) sv_topf(const __grid_constant__ TopfArgs g)
 {
     __shared__ float s_w[kTopfThreads];
     __shared__ int s_v[kTopfThreads];
