@@ -898,7 +898,7 @@ bool lr_shape_ok(int M, int d, int r, int V)
 }
 
 constexpr int kLrUpBN = 256;
-constexpr int kLrDownBN = 32;
+constexpr int kLrDownBN = 64;
 constexpr int kLrMaxSplits = 8;
 
 // K slices for the down contraction inside the head: enough CTAs to fill the SMs
