@@ -724,25 +724,32 @@ __global__ void __launch_bounds__(kPruneThreads) sv_tree_prune_rows(PruneArgs a)
     lse_init(L);
     Amax A{-INFINITY, 0x7fffffff, 0};
     constexpr int kPB = 4;  // groups per thread loaded before any is used
+    // the normaliser on packed fp32 pairs (one max and at most one rescale per
+    // batch, 8 accumulators folded at the end); groups past the row read as -inf
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint32_t ninf = ESZ == 2 ? 0xff80ff80u : 0xff800000u;
     for (long long g0 = tid; g0 < a.G; g0 += (long long)kPruneThreads * kPB) {
         uint4 raw[kPB];
 #pragma unroll
-        for (int u = 0; u < kPB; ++u)
-            if (g0 + (long long)kPruneThreads * u < a.G) raw[u] = tree_raw<ESZ, VEC16>(row, g0 + (long long)kPruneThreads * u, a.V);
-#pragma unroll
         for (int u = 0; u < kPB; ++u) {
             const long long g = g0 + (long long)kPruneThreads * u;
-            if (g >= a.G) break;
-            float x[VEC];
-            unpack<ESZ>(raw[u], x);
-            if (greedy) {
+            raw[u] = g < a.G ? tree_raw<ESZ, VEC16>(row, g, a.V) : make_uint4(ninf, ninf, ninf, ninf);
+        }
+        if (greedy) {
+#pragma unroll
+            for (int u = 0; u < kPB; ++u) {
+                const long long g = g0 + (long long)kPruneThreads * u;
+                if (g >= a.G) break;
+                float x[VEC];
+                unpack<ESZ>(raw[u], x);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) amax_add(A, x[e], (int)(g * VEC + e));
-            } else {
-                lse_add<VEC>(L, x, khi, klo);
             }
+        } else {
+            lse_group2<ESZ, kPB>(L, acc, raw, khi, klo);
         }
     }
+    if (!greedy) lse_fold(L, acc);
     const int nanf = __any_sync(0xffffffffu, L.s != L.s);
     lse_warp_merge(L);
     amax_warp_merge(A);
