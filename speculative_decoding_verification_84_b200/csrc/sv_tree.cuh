@@ -363,19 +363,18 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         const int nrows = kids ? 2 : 1;
         for (int r = 0; r < nrows; ++r) {
             const unsigned char* row = r == 0 ? trow : drow;
+            // packed fp32 pairs: one max and at most one rescale per batch, 8
+            // accumulators folded at the end; groups past the part read as -inf
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const uint32_t ninf = ESZ == 2 ? 0xff80ff80u : 0xff800000u;
             for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
                 uint4 raw[kTreeBatch];
 #pragma unroll
                 for (int u = 0; u < kTreeBatch; ++u)
-                    if (g0 + 32 * u < hi) raw[u] = tree_raw<ESZ, VEC16>(row, g0 + 32 * u, V);
-#pragma unroll
-                for (int u = 0; u < kTreeBatch; ++u)
-                    if (g0 + 32 * u < hi) {
-                        float x[VEC];
-                        unpack<ESZ>(raw[u], x);
-                        lse_add<VEC>(L[r], x, khi, klo);
-                    }
+                    raw[u] = g0 + 32 * u < hi ? tree_raw<ESZ, VEC16>(row, g0 + 32 * u, V) : make_uint4(ninf, ninf, ninf, ninf);
+                lse_group2<ESZ, kTreeBatch>(L[r], acc, raw, khi, klo);
             }
+            lse_fold(L[r], acc);
             // a NaN anywhere makes the thread's sum NaN; it is carried apart, since a
             // part whose maximum is -inf is dropped by the merges
             const int nanf = __any_sync(0xffffffffu, L[r].s != L[r].s);
