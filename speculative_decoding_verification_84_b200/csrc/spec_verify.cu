@@ -785,7 +785,7 @@ extern "C" sv_status spec_verify_tree_prune(const void* draft_logits, sv_dtype d
         else sv::sv_tree_prune_rows<4, false><<<grid, sv::kPruneThreads, 0, st>>>(g);
     }
     if (cudaGetLastError() != cudaSuccess) return SV_ERR_CUDA;
-    sv::sv_tree_prune_walk<<<(unsigned)cdiv(B, 128), 128, 0, st>>>(g);
+    sv::sv_tree_prune_walk<<<(unsigned)cdiv(B, sv::kWalkWarps), sv::kWalkWarps * 32, 0, st>>>(g);
     return cudaGetLastError() == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }
 

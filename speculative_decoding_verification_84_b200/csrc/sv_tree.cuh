@@ -223,6 +223,10 @@ struct TreeSmem {
     int next_sib[kTreeMaxNodes];
     int path[kTreeMaxNodes];
     float lt[kTreeMaxNodes], ld[kTreeMaxNodes];  // the children's logits at the current node
+    int pr[kTreeMaxNodes];            // the sequence's parent indices, tokens, keep flags and
+    int tk[kTreeMaxNodes];            // accept uniforms, loaded once by N threads at once
+    int kp[kTreeMaxNodes];
+    float ua[kTreeMaxNodes];
     int status;
 };
 
@@ -249,8 +253,6 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
     const size_t rowlen = (size_t)V * ESZ;
     const unsigned char* tgt = static_cast<const unsigned char*>(a.tgt) + (size_t)b * N * rowlen;
     const unsigned char* dft = static_cast<const unsigned char*>(a.dft) + (size_t)b * N * rowlen;
-    const int32_t* par = a.parent + (size_t)b * N;
-    const int32_t* tok = a.tokens + (size_t)b * N;
     const float T = a.temperature[b];
     const bool tval = temperature_ok(T), greedy = (T == 0.f);
     // this lane's groups of any row: g = lo + 32 j + lane, lo <= g < hi
@@ -259,7 +261,18 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
     const long long lo = min(cta_hi, cta0 + (long long)warp * a.GPW);
     const long long hi = min(cta_hi, lo + a.GPW);
 
-    // ---- the tree, the nodes that take part, the input checks (every CTA alike)
+    // ---- the tree, the nodes that take part, the input checks (every CTA alike);
+    // the per-node inputs first, one node per thread, so their loads overlap
+    if (tid < N) {
+        const size_t i = (size_t)b * N + tid;
+        sm.pr[tid] = a.parent[i];
+        sm.tk[tid] = a.tokens[i];
+        sm.kp[tid] = a.keep == nullptr ? 1 : a.keep[i];
+        sm.ua[tid] = a.u_accept[i];
+    }
+    __syncthreads();
+    const int* par = sm.pr;
+    const int* tok = sm.tk;
     if (tid == 0) {
         int st = 0;
         if (!tval) st = SV_ROW_BAD_TEMPERATURE;
@@ -271,11 +284,11 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         for (int i = 1; i < N; ++i) {
             const int p = par[i];
             if (p < 0 || p >= i) { st |= SV_ROW_BAD_TREE; sm.in[i] = 0; continue; }
-            sm.in[i] = sm.in[p] && (a.keep == nullptr || a.keep[(size_t)b * N + i] != 0);
+            sm.in[i] = sm.in[p] && sm.kp[i] != 0;
             if (!sm.in[i]) continue;
             if (tok[i] < 0 || tok[i] >= V) st |= SV_ROW_BAD_TOKEN;
             if (!greedy) {
-                const float u = a.u_accept[(size_t)b * N + i];
+                const float u = sm.ua[i];
                 if (!(u >= 0.f && u < 1.f)) st |= SV_ROW_BAD_UNIFORM;
             }
             if (last_child[p] < 0) sm.first_child[p] = i;
@@ -436,7 +449,7 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
             const double lq = (double)sm.ld[k] / Td - a2d * kLn2;
             const double lp = level == 0 ? (double)sm.lt[k] / Td - a2t * kLn2
                                          : log((double)tree_weight(rw, sm.inv_S, level, false, sm.lt[k], sm.ld[k]));
-            if (log((double)a.u_accept[(size_t)b * N + i]) < lp - lq) { next = i; break; }
+            if (log((double)sm.ua[i]) < lp - lq) { next = i; break; }
             // rejected: the mass of max(0, P - q)
             double part = 0.0;
             for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
@@ -679,13 +692,9 @@ struct PruneArgs {
     long long G;
 };
 
-__device__ __forceinline__ bool prune_seq_ok(const int32_t* par, int N, float T)
-{
-    if (!temperature_ok(T) || par[0] != -1) return false;
-    for (int i = 1; i < N; ++i)
-        if (par[i] < 0 || par[i] >= i) return false;
-    return true;
-}
+// A sequence takes part in pruning when its temperature is valid, parent[0] = -1
+// and 0 <= parent[i] < i for every other node (each lane checks its nodes).
+__device__ __forceinline__ bool prune_node_ok(int i, int p) { return i == 0 ? p == -1 : (p >= 0 && p < i); }
 
 // One CTA per (sequence b, node c) of a well-formed sequence in which c has
 // children: log q_c(tok_i) for every child i of c -- ld/T - lse(ld/T) of draft row
@@ -707,11 +716,18 @@ __global__ void __launch_bounds__(kPruneThreads) sv_tree_prune_rows(PruneArgs a)
     const int32_t* par = a.parent + (size_t)b * a.N;
     const int32_t* tok = a.tokens + (size_t)b * a.N;
     const float T = a.temperature[b];
-    if (tid == 0) {
-        int go = prune_seq_ok(par, a.N, T);
-        int kids = 0;
-        for (int i = c + 1; i < a.N && go; ++i) kids |= (par[i] == c);
-        s_go = go && kids;
+    if (warp == 0) {
+        // the sequence's tree is well formed and c has a child: one parent index
+        // per lane, all loads in flight at once
+        bool ok = temperature_ok(T), kid = false;
+        for (int i = lane; i < a.N; i += 32) {
+            const int p = par[i];
+            ok = ok && prune_node_ok(i, p);
+            kid = kid || (i > c && p == c);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        kid = __any_sync(0xffffffffu, kid);
+        if (lane == 0) s_go = ok && kid;
     }
     __syncthreads();
     if (!s_go) return;
@@ -784,26 +800,53 @@ __global__ void __launch_bounds__(kPruneThreads) sv_tree_prune_rows(PruneArgs a)
     }
 }
 
-// One thread per sequence: cum[i] = cum[parent] + log q, keep[i] = keep[parent]
-// and not (cum[i] < threshold), in node order (parents come first).  A sequence
-// with a bad temperature or tree keeps every node, with cum NaN.
-__global__ void sv_tree_prune_walk(PruneArgs a)
+// One warp per sequence: cum[i] = cum[parent] + log q, keep[i] = keep[parent]
+// and not (cum[i] < threshold), in node order (parents come first).  The parents
+// and log-probabilities are loaded by the lanes at once and walked in shared
+// memory by lane 0.  A sequence with a bad temperature or tree keeps every node,
+// with cum NaN.
+constexpr int kWalkWarps = 4;
+
+__global__ void __launch_bounds__(kWalkWarps * 32) sv_tree_prune_walk(PruneArgs a)
 {
-    const int b = (int)(blockIdx.x * blockDim.x + threadIdx.x);
-    if (b >= a.B) return;
-    const int32_t* par = a.parent + (size_t)b * a.N;
-    double* cum = a.out_cum + (size_t)b * a.N;
-    int32_t* keep = a.out_keep + (size_t)b * a.N;
-    if (!prune_seq_ok(par, a.N, a.temperature[b])) {
-        for (int i = 0; i < a.N; ++i) { keep[i] = 1; cum[i] = (double)NAN; }
+    __shared__ double s_cum[kWalkWarps][kTreeMaxNodes];
+    __shared__ int s_par[kWalkWarps][kTreeMaxNodes];
+    __shared__ int s_keep[kWalkWarps][kTreeMaxNodes];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = (int)blockIdx.x * kWalkWarps + warp;
+    if (b >= a.B) return;  // the whole warp
+    const int N = a.N;
+    const int32_t* par = a.parent + (size_t)b * N;
+    double* cum = a.out_cum + (size_t)b * N;
+    int32_t* keep = a.out_keep + (size_t)b * N;
+    bool ok = temperature_ok(a.temperature[b]);
+    for (int i = lane; i < N; i += 32) {
+        const int p = par[i];
+        s_par[warp][i] = p;
+        s_cum[warp][i] = cum[i];
+        ok = ok && prune_node_ok(i, p);
+    }
+    if (!__all_sync(0xffffffffu, ok)) {
+        for (int i = lane; i < N; i += 32) { keep[i] = 1; cum[i] = (double)NAN; }
         return;
     }
-    cum[0] = 0.0;
-    keep[0] = 1;
-    for (int i = 1; i < a.N; ++i) {
-        const int c = par[i];
-        cum[i] = cum[c] + cum[i];
-        keep[i] = keep[c] && !(cum[i] < a.threshold);
+    __syncwarp();
+    if (lane == 0) {
+        double* sc = s_cum[warp];
+        int* sk = s_keep[warp];
+        const int* sp = s_par[warp];
+        sc[0] = 0.0;
+        sk[0] = 1;
+        for (int i = 1; i < N; ++i) {
+            const int c = sp[i];
+            sc[i] = sc[c] + sc[i];
+            sk[i] = sk[c] && !(sc[i] < a.threshold);
+        }
+    }
+    __syncwarp();
+    for (int i = lane; i < N; i += 32) {
+        cum[i] = s_cum[warp][i];
+        keep[i] = s_keep[warp][i];
     }
 }
 
