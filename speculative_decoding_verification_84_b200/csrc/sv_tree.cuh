@@ -227,6 +227,11 @@ struct TreeSmem {
     int tk[kTreeMaxNodes];            // accept uniforms, loaded once by N threads at once
     int kp[kTreeMaxNodes];
     float ua[kTreeMaxNodes];
+    double lu[kTreeMaxNodes];         // log u_accept of each node
+    double nn_a2[2];                  // the current node's log2-normalisers (target, draft),
+    float nn_mk[2], nn_inv[2];        // offsets and reciprocal sums, folded by warp 0
+    int nn_bad;
+    int accept;                       // the current child's test, by thread 0
     int status;
 };
 
@@ -268,7 +273,9 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         sm.pr[tid] = a.parent[i];
         sm.tk[tid] = a.tokens[i];
         sm.kp[tid] = a.keep == nullptr ? 1 : a.keep[i];
-        sm.ua[tid] = a.u_accept[i];
+        const float u = a.u_accept[i];
+        sm.ua[tid] = u;
+        sm.lu[tid] = log((double)u);
     }
     __syncthreads();
     const int* par = sm.pr;
@@ -415,29 +422,41 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         }
         __syncthreads();
         tree_exchange(cl, sm, xpar, s_mine, CL, rank);
-        float Mr[2], MKr[2];
-        double Sr[2];
-        bool badr = false;
-        for (int r = 0; r < nrows; ++r) {
-            Mr[r] = -INFINITY; MKr[r] = 0.f; Sr[r] = 0.0;
-            for (int q = 0; q < CL; ++q) {
-                badr |= sm.x[xpar][q].bad[r] != 0;
-                lse_fold64(Mr[r], MKr[r], Sr[r], sm.x[xpar][q].m[r], sm.x[xpar][q].mk[r], sm.x[xpar][q].s[r]);
+        // the cluster's parts folded by warp 0 (lane r: row r, parts in rank order)
+        // and shared with the CTA
+        if (warp == 0) {
+            float Mq = -INFINITY, MKq = 0.f;
+            double Sq = 0.0;
+            bool bq = false;
+            if (lane < nrows) {
+                for (int q = 0; q < CL; ++q) {
+                    bq |= sm.x[xpar][q].bad[lane] != 0;
+                    lse_fold64(Mq, MKq, Sq, sm.x[xpar][q].m[lane], sm.x[xpar][q].mk[lane], sm.x[xpar][q].s[lane]);
+                }
+                bq |= (Mq == -INFINITY) || (Mq == INFINITY) || !isfinite(Sq) || !(Sq > 0.0);
             }
-            badr |= (Mr[r] == -INFINITY) || (Mr[r] == INFINITY) || !isfinite(Sr[r]) || !(Sr[r] > 0.0);
+            const bool bad_any = __any_sync(0xffffffffu, bq);
+            if (lane < 2) {
+                const bool use = lane < nrows && !bq;
+                sm.nn_a2[lane] = use ? (double)MKq + log2(Sq) : 0.0;
+                sm.nn_mk[lane] = use ? MKq : 0.f;
+                sm.nn_inv[lane] = use ? (float)(1.0 / Sq) : 0.f;
+            }
+            if (lane == 0) sm.nn_bad = bad_any;
         }
+        __syncthreads();
         xpar ^= 1;
-        if (badr) { st |= SV_ROW_BAD_LOGITS; break; }
-        const double a2t = (double)MKr[0] + log2(Sr[0]);
-        const double a2d = kids ? (double)MKr[1] + log2(Sr[1]) : 0.0;
+        if (sm.nn_bad) { st |= SV_ROW_BAD_LOGITS; break; }
+        const double a2t = sm.nn_a2[0];
+        const double a2d = kids ? sm.nn_a2[1] : 0.0;
         if (rank == 0 && tid == 0 && a.out_log_norm) {
             a.out_log_norm[(size_t)b * 2 * N + c] = a2t * kLn2;
             if (kids) a.out_log_norm[(size_t)b * 2 * N + N + c] = a2d * kLn2;
         }
         TreeRow rw;
         rw.khi = khi; rw.klo = klo;
-        rw.mk_t = MKr[0]; rw.inv_t = (float)(1.0 / Sr[0]);
-        rw.mk_d = kids ? MKr[1] : 0.f; rw.inv_d = kids ? (float)(1.0 / Sr[1]) : 0.f;
+        rw.mk_t = sm.nn_mk[0]; rw.inv_t = sm.nn_inv[0];
+        rw.mk_d = kids ? sm.nn_mk[1] : 0.f; rw.inv_d = kids ? sm.nn_inv[1] : 0.f;
 
         // ---- the children, in index order
         const double Td = (double)T;
@@ -446,10 +465,15 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
         // weights are that residual, so its sums (sm.wsum, sm.x[reuse_par]) stand
         int reuse_par = -1;
         for (int i = sm.first_child[c]; i >= 0; i = sm.next_sib[i], ++k) {
-            const double lq = (double)sm.ld[k] / Td - a2d * kLn2;
-            const double lp = level == 0 ? (double)sm.lt[k] / Td - a2t * kLn2
-                                         : log((double)tree_weight(rw, sm.inv_S, level, false, sm.lt[k], sm.ld[k]));
-            if (log((double)sm.ua[i]) < lp - lq) { next = i; break; }
+            // the test, by one thread for the CTA
+            if (tid == 0) {
+                const double lq = (double)sm.ld[k] / Td - a2d * kLn2;
+                const double lp = level == 0 ? (double)sm.lt[k] / Td - a2t * kLn2
+                                             : log((double)tree_weight(rw, sm.inv_S, level, false, sm.lt[k], sm.ld[k]));
+                sm.accept = sm.lu[i] < lp - lq;
+            }
+            __syncthreads();
+            if (sm.accept) { next = i; break; }
             // rejected: the mass of max(0, P - q)
             double part = 0.0;
             for (long long g0 = lo + lane; g0 < hi; g0 += 32 * kTreeBatch) {
