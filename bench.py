@@ -144,7 +144,9 @@ def job_value(local_ms, world, per_rank_units, pg=None, device=None):
 
 
 def oracle_time(w, min_seconds, n_threads=0):
-    """Time the oracle on the batch, repeated until min_seconds of CPU work; seq-steps/s."""
+    """Time the oracle on the batch, repeated until min_seconds of CPU work; seq-steps/s.
+    n_threads > 0 sets the oracle's OpenMP thread count for the rest of the process,
+    so the one-core sample is taken last."""
     import oracle
     oracle.build()
     cores = n_threads or oracle.max_threads()
@@ -789,6 +791,10 @@ def run_ours(args):
         val, cores, reps, el = oracle_time(w, args.cpu_seconds)
         cpu = {"value": val, "unit": "seq-steps/s", "cores": cores, "kind": "oracle",
                "sample": f"{reps} passes over the full c3 batch ({w.B} sequences), {el:.1f} s, fp64 C oracle"}
+        # the same oracle on one core, a shorter sample
+        v1, _, r1, e1 = oracle_time(w, min(3.0, args.cpu_seconds), n_threads=1)
+        cpu["one_core"] = {"value": v1, "unit": "seq-steps/s", "cores": 1,
+                           "sample": f"{r1} passes over the full c3 batch, {e1:.1f} s"}
 
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
