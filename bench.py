@@ -889,6 +889,14 @@ def run_profile(args):
         torch.cuda.synchronize()
         print(f"t3: {args.warmup + args.steps} calls, 1 launch each", flush=True)
         return 0
+    if args.profile == "t3prune":
+        w = W.make_tree(64, TREE_SHAPE, 128256, "bf16", seed=91, name="t3")
+        d = binding.tree_to_device(w, "cuda:0")
+        for i in range(args.warmup + args.steps):
+            binding.tree_prune(d["draft"], d["parent"], d["tokens"], d["temperature"], -12.0)
+        torch.cuda.synchronize()
+        print(f"t3prune: {args.warmup + args.steps} calls, 2 launches each", flush=True)
+        return 0
     c = Caller(W.make_workload(args.profile), torch.device("cuda", 0), lib, binding)
     for i in range(args.warmup + args.steps):
         c.call(i)
@@ -906,7 +914,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="skip the line's per-workload numbers")
-    ap.add_argument("--profile", choices=list(PER_CONFIG) + ["t3", "h3", "c3topf", "bandit"], default=None,
+    ap.add_argument("--profile", choices=list(PER_CONFIG) + ["t3", "t3prune", "h3", "c3topf", "bandit"], default=None,
                     help="only make warm-up + K calls of this workload (for a profiler); no JSON line")
     args = ap.parse_args()
     if args.profile:
