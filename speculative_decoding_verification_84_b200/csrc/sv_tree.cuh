@@ -637,6 +637,14 @@ __global__ void __launch_bounds__(kTreeThreads, 2) sv_tree(TreeArgs a)
             const int ws = s_found;
             int tokf = -1;
             if (ws >= 0 && warp == ws) {
+                // the warp's groups into L1 first (from L2, where the passes left
+                // them), so the walk below does not wait on L2 once per block
+                if constexpr (VEC16) {
+                    for (long long g = lo + lane; g < hi; g += 32) {
+                        asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint4*>(trow) + g));
+                        if (resid) asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint4*>(drow) + g));
+                    }
+                }
                 double C = sm.wsum[0];
                 for (long long gb = lo; gb < hi && tokf < 0; gb += 32) {
                     const long long g = gb + lane;
