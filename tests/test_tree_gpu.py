@@ -145,3 +145,33 @@ def test_tree_edge_cases():
     assert st[3] in (0, 8) and st[7] in (0, 8) and st[10] in (0, 8) and st[13] == 0
     sure = r.near_tie == 0
     assert (toks[sure] == r.out_tokens[sure]).all() and (n[sure] == r.n_accepted[sure]).all()
+
+
+def test_tree_prune_edge_cases():
+    """Pruning on malformed sequences: a bad parent index, a node after its own
+    index, a bad or NaN temperature (every node kept, cum NaN); a token outside
+    [0, V) and a NaN draft row on a kept path (NaN entries, nodes kept); greedy and
+    ragged rows (scalar loads); every output equal to the oracle's."""
+    for V, dt in ((300, "f32"), (333, "bf16"), (4096, "bf16")):
+        w = W.make_tree(10, (2, 2), V, dt, seed=17 + V, T=[1.0, 0.7, 0.0, 1.3, 1.0, 1.0, 0.0, 1.0, 1.0, 2.0])
+        par, tok, dft, T = w.parent.copy(), w.tokens.copy(), w.draft.copy(), w.temperature.copy()
+        par[0, 3] = 3                 # a node its own parent
+        par[1, 0] = 0                 # the root with a parent
+        T[4] = -1.0                   # bad temperature
+        T[5] = np.nan
+        tok[7, 2] = V                 # a token outside the vocabulary
+        dft[8, 1] = np.nan if dt == "f32" else 0x7fc0  # a NaN row with children
+        we = W.TreeWorkload("prune_edges", dt, w.target, dft, par, tok, T, w.u_accept, w.u_resample)
+        d = binding.tree_to_device(we, DEV)
+        for thr in (-np.inf, -9.0):
+            keep, cum = binding.tree_prune(d["draft"], d["parent"], d["tokens"], d["temperature"], thr)
+            keep, cum = keep.cpu().numpy(), cum.cpu().numpy()
+            ek, ec = oracle.tree_prune(dft, par, tok, T, thr, bf16=(dt == "bf16"))
+            assert (np.isnan(cum) == np.isnan(ec)).all(), (V, thr)
+            fin = np.isfinite(ec)
+            assert (np.isneginf(cum) == np.isneginf(ec)).all()
+            assert np.allclose(cum[fin], ec[fin], rtol=1e-9, atol=1e-6), (V, thr)
+            clear = ~(np.abs(np.where(fin, ec, 0.0) - (thr if np.isfinite(thr) else 0.0)) < 1e-5)
+            assert (keep[clear] == ek[clear]).all(), (V, thr)
+            for b in (0, 1, 4, 5):
+                assert (keep[b] == 1).all() and np.isnan(cum[b]).all(), (V, b)
