@@ -27,12 +27,15 @@
 //                   distributed shared memory: every CTA pushes its part into
 //                   every CTA's buffer, one cluster barrier, and every CTA folds
 //                   the parts in rank order -- so every CTA takes the same
-//                   decisions and no further broadcast is needed.  Only the rows
-//                   of the nodes the walk visits are read.
+//                   decisions and no further broadcast is needed.  Inside a CTA
+//                   the scalar work (the folds, the tests) is done once, by warp
+//                   0 or thread 0, and shared through shared memory.  Only the
+//                   rows of the nodes the walk visits are read.
 //   sv_tree_prune_rows / sv_tree_prune_walk
 //                   the draft's log q_c(tok_i) for every node i with parent c
 //                   (one CTA per (sequence, parent row)), then the cumulative
-//                   sums and the keep mask along the parent order.
+//                   sums and the keep mask along the parent order (one warp per
+//                   sequence, in shared memory).
 #pragma once
 
 #include <cooperative_groups.h>
